@@ -1,0 +1,300 @@
+"""CPU oracle for the block-scaled W8A8 linear layer and its MoE variant.
+
+TEST INFRASTRUCTURE ONLY: the test-suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are its only users.  The product path (the
+CUDA library and its Python binding) never imports this package, and this
+package imports nothing from the product path.
+
+The arithmetic lives in ``bq_oracle.c`` (plain C, fp64, compiled with gcc
+without fast-math).  This module compiles it on first use and wraps each
+function for numpy arrays.  Layout conventions here are the natural ones:
+activation scales are ``[M, Kb]`` and weight scales ``[Nb, Kb]``, row-major.
+
+Sources are cited in ``bq_oracle.c``; in short:
+  * block-wise INT8 page ("[SGLang] Block-wise INT8"): weight layout and scale
+    grid (structure diagram, section 2), dynamic activation quantisation
+    (section 4), MoE gate+up fused weights (section 5), int8 range (design
+    rationale item 3);
+  * SGLang quantization doc, "GEMM backends for FP4/FP8": blockwise FP8;
+  * "LLM quantization overview" page, FP8 section: e4m3 bit layout.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+INT8 = 0
+FP8 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_bq_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# gcc flags: IEEE semantics, no fast-math, no FTZ.
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off"]
+
+
+def build(force: bool = False) -> str:
+    """Compile bq_oracle.c into _bq_oracle.so next to it (if stale)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    P, L, I, D = ctypes.c_void_p, ctypes.c_long, ctypes.c_int, ctypes.c_double
+    lib.bq_ref_bf16_to_double.argtypes = [ctypes.c_uint16]
+    lib.bq_ref_bf16_to_double.restype = D
+    lib.bq_ref_bf16_from_double.argtypes = [D]
+    lib.bq_ref_bf16_from_double.restype = ctypes.c_uint16
+    lib.bq_ref_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.bq_ref_e4m3_decode.restype = D
+    lib.bq_ref_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.bq_ref_e4m3_encode.restype = ctypes.c_uint8
+    lib.bq_ref_quant_act.argtypes = [P, L, L, L, L, I, P, L, P]
+    lib.bq_ref_quant_act.restype = None
+    lib.bq_ref_quant_weight.argtypes = [P, L, L, L, L, L, I, P, L, P]
+    lib.bq_ref_quant_weight.restype = None
+    lib.bq_ref_gemm_entry.argtypes = [P, L, P, P, L, P, L, L, L, L, L, I, P, L, L]
+    lib.bq_ref_gemm_entry.restype = D
+    lib.bq_ref_gemm.argtypes = [P, L, P, P, L, P, L, L, L, L, L, L, I, P, P]
+    lib.bq_ref_gemm.restype = None
+    lib.bq_ref_dequant_dot.argtypes = [P, L, P, P, L, P, L, L, L, L, L, I, L, L]
+    lib.bq_ref_dequant_dot.restype = D
+    lib.bq_ref_moe_permute.argtypes = [P, L, L, L, P, P, P]
+    lib.bq_ref_moe_permute.restype = I
+    lib.bq_ref_silu_mul.argtypes = [P, L, L, L, P]
+    lib.bq_ref_silu_mul.restype = None
+    lib.bq_ref_moe_combine.argtypes = [P, L, P, P, L, L, L, P]
+    lib.bq_ref_moe_combine.restype = None
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = configure(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def cdiv(a: int, b: int) -> int:
+    """Ceil division, the scale-grid rule of the block-wise INT8 page, section 2."""
+    return (a + b - 1) // b
+
+
+# --------------------------------------------------------------------------
+# scalar helpers
+# --------------------------------------------------------------------------
+
+def bf16_to_f64(h) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64 values."""
+    h = np.asarray(h, dtype=np.uint16)
+    u = h.astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def bf16_from_f64(v) -> np.ndarray:
+    """Round float64 values once to bf16 (RNE); returns uint16 bit patterns."""
+    lib = _load()
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    flat_in, flat_out = v.reshape(-1), out.reshape(-1)
+    for i in range(flat_in.size):
+        flat_out[i] = lib.bq_ref_bf16_from_double(float(flat_in[i]))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    lib = _load()
+    c = np.asarray(c, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    fi, fo = c.reshape(-1), out.reshape(-1)
+    for i in range(fi.size):
+        fo[i] = lib.bq_ref_e4m3_decode(int(fi[i]))
+    return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    lib = _load()
+    x = np.asarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    fi, fo = x.reshape(-1), out.reshape(-1)
+    for i in range(fi.size):
+        fo[i] = lib.bq_ref_e4m3_encode(float(fi[i]))
+    return out
+
+
+def code_values(q: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact values of stored codes (raw bytes)."""
+    q = np.asarray(q, dtype=np.uint8)
+    if dtype == INT8:
+        return q.view(np.int8).astype(np.float64)
+    table = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return table[q]
+
+
+# --------------------------------------------------------------------------
+# a1 / a2: quantisation
+# --------------------------------------------------------------------------
+
+def quant_act(x_bf16: np.ndarray, group_k: int, dtype: int):
+    """Dynamic 1 x group_k activation quantisation.
+
+    x_bf16: uint16 [M, K] bf16 bit patterns.  Returns (q uint8 [M, K],
+    s float32 [M, Kb])."""
+    lib = _load()
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    Kb = cdiv(K, group_k)
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty((M, Kb), dtype=np.float32)
+    lib.bq_ref_quant_act(_ptr(x), M, K, K, group_k, dtype, _ptr(q), K, _ptr(s))
+    return q, s
+
+
+def quant_weight(w: np.ndarray, bn: int, bk: int, dtype: int):
+    """Offline [bn, bk] block quantisation of fp32 W [N, K].
+
+    Returns (q uint8 [N, K], s float32 [ceil(N/bn), ceil(K/bk)])."""
+    lib = _load()
+    w = _c(w, np.float32)
+    N, K = w.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    s = np.empty((cdiv(N, bn), cdiv(K, bk)), dtype=np.float32)
+    lib.bq_ref_quant_weight(_ptr(w), N, K, K, bn, bk, dtype, _ptr(q), K, _ptr(s))
+    return q, s
+
+
+def quant_weight_gate_up(w13: np.ndarray, I: int, bn: int, bk: int, dtype: int):
+    """Fused gate+up weight [2I, K]: the gate half [0, I) and the up half
+    [I, 2I) are blocked separately, so the scale grid has 2*ceil(I/bn) rows
+    (block-wise INT8 page, section 5)."""
+    q1, s1 = quant_weight(w13[:I], bn, bk, dtype)
+    q2, s2 = quant_weight(w13[I:], bn, bk, dtype)
+    return np.concatenate([q1, q2], 0), np.concatenate([s1, s2], 0)
+
+
+# --------------------------------------------------------------------------
+# a3 / a4: GEMM
+# --------------------------------------------------------------------------
+
+def gemm(qa, sa, qw, sw, bn: int, bk: int, dtype: int, bias_bf16=None, seam: int = 0):
+    """out64 [M, N] = sum_kb P_kb * sa[m,kb] * sw[nb(n),kb] (+ bias), fp64."""
+    lib = _load()
+    qa, qw = _c(qa, np.uint8), _c(qw, np.uint8)
+    sa, sw = _c(sa, np.float32), _c(sw, np.float32)
+    M, K = qa.shape
+    N = qw.shape[0]
+    bias = None if bias_bf16 is None else _c(bias_bf16, np.uint16)
+    out = np.empty((M, N), dtype=np.float64)
+    lib.bq_ref_gemm(_ptr(qa), K, _ptr(sa), _ptr(qw), K, _ptr(sw), M, N, K, bn, bk, seam,
+                    dtype, _ptr(bias), _ptr(out))
+    return out
+
+
+def gemm_entries(qa, sa, qw, sw, bn: int, bk: int, dtype: int, rows, cols,
+                 bias_bf16=None, seam: int = 0):
+    """Selected outputs out64[rows[i], cols[i]], computed one by one."""
+    lib = _load()
+    qa, qw = _c(qa, np.uint8), _c(qw, np.uint8)
+    sa, sw = _c(sa, np.float32), _c(sw, np.float32)
+    K = qa.shape[1]
+    N = qw.shape[0]
+    bias = None if bias_bf16 is None else _c(bias_bf16, np.uint16)
+    res = np.empty(len(rows), dtype=np.float64)
+    for i, (m, n) in enumerate(zip(rows, cols)):
+        res[i] = lib.bq_ref_gemm_entry(_ptr(qa), K, _ptr(sa), _ptr(qw), K, _ptr(sw), N, K,
+                                       bn, bk, seam, dtype, _ptr(bias), int(m), int(n))
+    return res
+
+
+def dequant_dot(qa, sa, qw, sw, bn: int, bk: int, dtype: int, m: int, n: int,
+                seam: int = 0) -> float:
+    lib = _load()
+    qa, qw = _c(qa, np.uint8), _c(qw, np.uint8)
+    sa, sw = _c(sa, np.float32), _c(sw, np.float32)
+    K = qa.shape[1]
+    N = qw.shape[0]
+    return lib.bq_ref_dequant_dot(_ptr(qa), K, _ptr(sa), _ptr(qw), K, _ptr(sw), N, K, bn, bk,
+                                  seam, dtype, m, n)
+
+
+# --------------------------------------------------------------------------
+# a5-a9: MoE
+# --------------------------------------------------------------------------
+
+def moe_permute(ids: np.ndarray, E: int):
+    """Stable expert-major order of the (token, slot) pairs.
+
+    Returns (offsets int32 [E+1], perm int32 [T*topk], inv_perm int32 [T*topk])."""
+    lib = _load()
+    ids = _c(ids, np.int32)
+    T, topk = ids.shape
+    R = T * topk
+    off = np.empty(E + 1, dtype=np.int32)
+    perm = np.empty(R, dtype=np.int32)
+    inv = np.empty(R, dtype=np.int32)
+    rc = lib.bq_ref_moe_permute(_ptr(ids), T, topk, E, _ptr(off), _ptr(perm), _ptr(inv))
+    if rc != 0:
+        raise ValueError("expert id out of range")
+    return off, perm, inv
+
+
+def silu_mul(y_bf16: np.ndarray, I: int):
+    """h = bf16(silu(gate) * up) with gate = y[:, :I], up = y[:, I:2I]."""
+    lib = _load()
+    y = _c(y_bf16, np.uint16)
+    R = y.shape[0]
+    h = np.empty((R, I), dtype=np.uint16)
+    lib.bq_ref_silu_mul(_ptr(y), R, I, y.shape[1], _ptr(h))
+    return h
+
+
+def moe_combine(y_bf16: np.ndarray, inv_perm: np.ndarray, w: np.ndarray):
+    """out[t] = bf16(sum_j w[t,j] * y[inv_perm[t*topk+j]]), fp64."""
+    lib = _load()
+    y = _c(y_bf16, np.uint16)
+    w = _c(w, np.float32)
+    inv = _c(inv_perm, np.int32)
+    T, topk = w.shape
+    H = y.shape[1]
+    out = np.empty((T, H), dtype=np.uint16)
+    lib.bq_ref_moe_combine(_ptr(y), H, _ptr(inv), _ptr(w), T, topk, H, _ptr(out))
+    return out
+
+
+def grouped_gemm(qa, sa, offsets, qw_e, sw_e, bn: int, bk: int, dtype: int, seam: int = 0):
+    """Per expert e, rows [offsets[e], offsets[e+1]) of qa against qw_e[e]."""
+    R = qa.shape[0]
+    N = qw_e.shape[1]
+    out = np.empty((R, N), dtype=np.float64)
+    for e in range(len(offsets) - 1):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 > r0:
+            out[r0:r1] = gemm(qa[r0:r1], sa[r0:r1], qw_e[e], sw_e[e], bn, bk, dtype,
+                              seam=seam)
+    return out

@@ -1,0 +1,242 @@
+// quant.cu -- activation and weight quantisation kernels.
+//
+// Activation quantisation (block-wise INT8 page, section 4: the activation
+// scale is computed at run time, per token, inside the kernel): each 1 x
+// group_k group of a row gets s = amax / Q and codes q = code(x / s).
+// One warp per group; for group_k <= 128 every lane holds its (up to) four
+// elements in registers, loaded as one 8-byte vector when aligned, and the
+// amax is a 5-step shuffle reduction.  Consecutive warps take consecutive
+// rows of the same K-block so the K-block-major scale stores coalesce.
+//
+// Weight quantisation (structure diagram and section 2): one CTA per
+// [bn, bk] block; amax by a block reduction, then codes.
+#include <algorithm>
+
+#include "bq_common.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+
+namespace {
+
+constexpr int kWarpsPerCta = 8;
+
+// Loads the (up to 4) elements [k0, k0+4) of a row restricted to [0, L).
+__device__ __forceinline__ void load4(const uint16_t* row, int64_t k0, int64_t L, bool vec,
+                                      float v[4]) {
+  if (vec && k0 + 4 <= L) {
+    uint2 u = *reinterpret_cast<const uint2*>(row + k0);
+    v[0] = bf16_bits_to_float((uint16_t)(u.x & 0xFFFFu));
+    v[1] = bf16_bits_to_float((uint16_t)(u.x >> 16));
+    v[2] = bf16_bits_to_float((uint16_t)(u.y & 0xFFFFu));
+    v[3] = bf16_bits_to_float((uint16_t)(u.y >> 16));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = (k0 + i < L) ? bf16_bits_to_float(row[k0 + i]) : 0.0f;
+  }
+}
+
+__device__ __forceinline__ void store4(uint8_t* row, int64_t k0, int64_t L, bool vec,
+                                       uint32_t w) {
+  if (vec && k0 + 4 <= L) {
+    *reinterpret_cast<uint32_t*>(row + k0) = w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (k0 + i < L) row[k0 + i] = (uint8_t)(w >> (8 * i));
+  }
+}
+
+// Source of the elements of one group: either a bf16 row, or (SILU) the
+// gate/up halves of a bf16 row combined as bf16(silu(g) * u).
+template <bool SILU>
+struct RowSource {
+  const uint16_t* row;   // start of the group (gate half for SILU)
+  const uint16_t* up;    // SILU only: start of the group in the up half
+  uint16_t* h_out;       // SILU only: optional bf16 copy of h
+  bool vec;
+  __device__ __forceinline__ void get4(int64_t k0, int64_t L, float v[4]) const {
+    if (!SILU) {
+      load4(row, k0, L, vec, v);
+    } else {
+      float g[4], u[4];
+      load4(row, k0, L, vec, g);
+      load4(up, k0, L, vec, u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // silu(g) = g / (1 + exp(-g)) in fp32, times u, rounded once to bf16
+        float sg = __fdiv_rn(g[i], 1.0f + expf(-g[i]));
+        uint16_t hb = float_to_bf16_bits(sg * u[i]);
+        v[i] = (k0 + i < L) ? bf16_bits_to_float(hb) : 0.0f;
+      }
+      if (h_out) {
+        if (vec && k0 + 4 <= L) {
+          uint2 w;
+          w.x = (uint32_t)float_to_bf16_bits(v[0]) | ((uint32_t)float_to_bf16_bits(v[1]) << 16);
+          w.y = (uint32_t)float_to_bf16_bits(v[2]) | ((uint32_t)float_to_bf16_bits(v[3]) << 16);
+          *reinterpret_cast<uint2*>(h_out + k0) = w;
+        } else {
+          for (int i = 0; i < 4; ++i)
+            if (k0 + i < L) h_out[k0 + i] = float_to_bf16_bits(v[i]);
+        }
+      }
+    }
+  }
+};
+
+// One warp quantises one group.  Groups of <= 128 elements stay in
+// registers (one read); longer groups are read twice (amax, then codes).
+template <int DT, bool SILU>
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+quant_rows_kernel(const uint16_t* __restrict__ x, int64_t M_out, int64_t K, int64_t ldx,
+                  const int32_t* __restrict__ perm, int64_t topk, int64_t gk, int64_t I_half,
+                  uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
+                  uint16_t* __restrict__ h_out, bool vec_in, bool vec_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t Kb = (K + gk - 1) / gk;
+  const int64_t n_groups = M_out * Kb;
+  const int64_t warp0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const int64_t wstride = (int64_t)gridDim.x * kWarpsPerCta;
+  for (int64_t w = warp0; w < n_groups; w += wstride) {
+    const int64_t g = w / M_out, m = w - g * M_out;
+    const int64_t src = perm ? (int64_t)perm[m] / topk : m;
+    const int64_t k0 = g * gk;
+    const int64_t L = min(gk, K - k0);
+    RowSource<SILU> srcrow;
+    srcrow.row = x + src * ldx + k0;
+    srcrow.up = SILU ? x + src * ldx + I_half + k0 : nullptr;
+    srcrow.h_out = (SILU && h_out) ? h_out + m * K + k0 : nullptr;
+    srcrow.vec = vec_in;
+    uint8_t* qrow = q + m * ldq + k0;
+    if (gk <= 128) {
+      float v[4];
+      srcrow.get4(4 * lane, L, v);
+      float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+      amax = warp_max(amax);
+      const float sc = group_scale<DT>(amax);
+      if (4 * lane < L) store4(qrow, 4 * lane, L, vec_out, pack4_codes<DT>(v, sc));
+      if (lane == 0) s[g * M_out + m] = sc;
+    } else {
+      float amax = 0.0f;
+      for (int64_t k = 4 * lane; k < L; k += 128) {
+        float v[4];
+        if (SILU) {
+          // h is only materialised in the second pass
+          RowSource<SILU> tmp = srcrow;
+          tmp.h_out = nullptr;
+          tmp.get4(k, L, v);
+        } else {
+          srcrow.get4(k, L, v);
+        }
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+      }
+      amax = warp_max(amax);
+      const float sc = group_scale<DT>(amax);
+      for (int64_t k = 4 * lane; k < L; k += 128) {
+        float v[4];
+        srcrow.get4(k, L, v);
+        store4(qrow, k, L, vec_out, pack4_codes<DT>(v, sc));
+      }
+      if (lane == 0) s[g * M_out + m] = sc;
+    }
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(256)
+quant_weight_kernel(const float* __restrict__ w, int64_t N, int64_t K, int64_t ldw, int64_t bn,
+                    int64_t bk, uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ s) {
+  __shared__ float red[8];
+  const int64_t Kb = (K + bk - 1) / bk;
+  const int64_t i = blockIdx.y, j = blockIdx.x;
+  const int64_t n0 = i * bn, k0 = j * bk;
+  const int64_t Ln = min(bn, N - n0), Lk = min(bk, K - k0);
+  const int64_t cnt = Ln * Lk;
+  float amax = 0.0f;
+  for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+    int64_t r = e / Lk, c = e - r * Lk;
+    amax = fmaxf(amax, fabsf(w[(n0 + r) * ldw + k0 + c]));
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float sc = group_scale<DT>(red[0]);
+  for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+    int64_t r = e / Lk, c = e - r * Lk;
+    q[(n0 + r) * ldq + k0 + c] = one_code<DT>(w[(n0 + r) * ldw + k0 + c], sc);
+  }
+  if (threadIdx.x == 0) s[i * Kb + j] = sc;
+}
+
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int grid_for_groups(int64_t n_groups) {
+  int64_t ctas = (n_groups + kWarpsPerCta - 1) / kWarpsPerCta;
+  const int64_t cap = 148 * 16;  // persistent-style cap: 16 CTAs per SM
+  return (int)std::max<int64_t>(1, std::min<int64_t>(ctas, cap));
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const void* x, int64_t M_out, int64_t K, int64_t ldx,
+                             const int32_t* perm, int64_t topk, int64_t group_k, int dtype,
+                             void* q, int64_t ldq, float* s, cudaStream_t st) {
+  if (M_out == 0 || K == 0) return cudaSuccess;
+  const int64_t Kb = (K + group_k - 1) / group_k;
+  const bool vec_in = aligned(x, 8) && ldx % 4 == 0 && group_k % 4 == 0;
+  const bool vec_out = aligned(q, 4) && ldq % 4 == 0 && group_k % 4 == 0;
+  const int grid = grid_for_groups(M_out * Kb);
+  auto xs = static_cast<const uint16_t*>(x);
+  auto qs = static_cast<uint8_t*>(q);
+  if (dtype == kInt8)
+    quant_rows_kernel<kInt8, false><<<grid, kWarpsPerCta * 32, 0, st>>>(
+        xs, M_out, K, ldx, perm, topk, group_k, 0, qs, ldq, s, nullptr, vec_in, vec_out);
+  else
+    quant_rows_kernel<kFp8, false><<<grid, kWarpsPerCta * 32, 0, st>>>(
+        xs, M_out, K, ldx, perm, topk, group_k, 0, qs, ldq, s, nullptr, vec_in, vec_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_silu_mul_quant(const void* y, int64_t ldy, int64_t R, int64_t I,
+                                  int64_t group_k, int dtype, void* q, int64_t ldq, float* s,
+                                  void* h_out, cudaStream_t st) {
+  if (R == 0 || I == 0) return cudaSuccess;
+  const int64_t Kb = (I + group_k - 1) / group_k;
+  const bool vec_in = aligned(y, 8) && ldy % 4 == 0 && group_k % 4 == 0 && I % 4 == 0 &&
+                      (h_out == nullptr || aligned(h_out, 8));
+  const bool vec_out = aligned(q, 4) && ldq % 4 == 0 && group_k % 4 == 0;
+  const int grid = grid_for_groups(R * Kb);
+  auto ys = static_cast<const uint16_t*>(y);
+  auto qs = static_cast<uint8_t*>(q);
+  auto hs = static_cast<uint16_t*>(h_out);
+  if (dtype == kInt8)
+    quant_rows_kernel<kInt8, true><<<grid, kWarpsPerCta * 32, 0, st>>>(
+        ys, R, I, ldy, nullptr, 1, group_k, I, qs, ldq, s, hs, vec_in, vec_out);
+  else
+    quant_rows_kernel<kFp8, true><<<grid, kWarpsPerCta * 32, 0, st>>>(
+        ys, R, I, ldy, nullptr, 1, group_k, I, qs, ldq, s, hs, vec_in, vec_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_weight(const float* w, int64_t N, int64_t K, int64_t ldw,
+                                int64_t bn, int64_t bk, int dtype, void* q, int64_t ldq,
+                                float* s, cudaStream_t st) {
+  if (N == 0 || K == 0) return cudaSuccess;
+  const int64_t Nb = (N + bn - 1) / bn, Kb = (K + bk - 1) / bk;
+  if (Nb > 65535) return cudaErrorInvalidConfiguration;
+  dim3 grid((unsigned)Kb, (unsigned)Nb);
+  auto qs = static_cast<uint8_t*>(q);
+  if (dtype == kInt8)
+    quant_weight_kernel<kInt8><<<grid, 256, 0, st>>>(w, N, K, ldw, bn, bk, qs, ldq, s);
+  else
+    quant_weight_kernel<kFp8><<<grid, 256, 0, st>>>(w, N, K, ldw, bn, bk, qs, ldq, s);
+  return cudaGetLastError();
+}
+
+}  // namespace bq

@@ -1,0 +1,273 @@
+/*
+ * bq.h -- C ABI of libbq: block-scaled W8A8 (INT8 / FP8-e4m3) linear layers
+ * and their MoE grouped-GEMM variant, for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources are web pages, cited by title and section):
+ *
+ *  - "[SGLang] Block-wise INT8: 블록 단위 정수 양자화" (the block-wise INT8 page):
+ *      structure diagram + section 2: weight W [N, K] int8 (row n = output
+ *        channel, K contiguous) with fp32 block scales [ceil(N/bn), ceil(K/bk)],
+ *        one per [block_n, block_k] block; the stored scale multiplies the
+ *        code back to the weight (W ~= q * s);
+ *      section 1: block size has two dimensions, activations are quantised
+ *        dynamically only, the checkpoint is already int8-serialised;
+ *      section 4: the activation scale is computed at run time (input_scale
+ *        = None), per token, inside the kernel;
+ *      section 5/6: MoE experts hold their own weights and scales; w13 is the
+ *        gate and up projections fused, [E, 2I, H], scales
+ *        [E, 2*ceil(I/bn), ceil(H/bk)].
+ *  - SGLang "양자화 (Quantization)" doc, "FP4/FP8 양자화용 GEMM 백엔드":
+ *      blockwise FP8 GEMM, the same contraction on e4m3 codes.
+ *  - "LLM 양자화 완전 정리 — FP8, AWQ, GPTQ, GGUF 차이와 선택법", FP8 section:
+ *      e4m3 = 1 sign, 4 exponent, 3 mantissa bits.
+ *
+ * The arithmetic, with the readings taken where the pages are silent:
+ *   activation group = 1 x group_k elements of one row (per token, per K-block);
+ *   s = amax / Q in IEEE fp32 division, Q = 127 (INT8) or 448 (FP8 e4m3);
+ *   q = clamp(round_half_even(x / s), -128, 127)           (INT8)
+ *     = e4m3(x / s), round-to-nearest-even, saturating at +-448  (FP8)
+ *     with x / s one IEEE fp32 division; an all-zero group has s = 0, q = 0;
+ *   out[m, n] = bf16( sum_kb P_kb[m,n] * sa[kb][m] * sw[nb(n)][kb] + bias[n] )
+ *     with P_kb the exact int32 (INT8) / fp32-accumulated (FP8) dot product
+ *     of the codes inside K-block kb, the sum over blocks in fp32, and one
+ *     round-to-nearest-even conversion to bf16 at the end.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller, except where
+ *    stated.  The library never allocates or frees device memory; kernels that
+ *    need scratch take a caller-provided workspace, sized by the matching
+ *    *_workspace_size query.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call only enqueues work on it and never synchronises, except
+ *    bq_check_device_status.
+ *  - Sizes are int64_t element counts; leading dimensions ("ld") are in
+ *    elements of the array's type.  bf16 arrays are passed as void* holding
+ *    16-bit bfloat16 values.  Quantised codes are passed as void* holding one
+ *    byte per element (int8 two's complement, or e4m3 bits).
+ *  - Every call returns a bq_status.  Argument errors are detected on the host
+ *    before anything is enqueued; bq_last_error_message() then describes the
+ *    problem (thread-local).  M == 0 (or N == 0, R == 0, T == 0) is a no-op.
+ *  - Activation scales use the K-block-major layout [Kb][M] (Kb =
+ *    ceil(K/group_k)), dense: the scale of row m in K-block g is s[g*M + m].
+ *    (The pages do not fix this layout; K-block-major lets a GEMM tile read
+ *    the scales of its rows for one K-block as one contiguous run.)
+ *  - Weight scales are [Nb][Kb] row-major as on the block-wise INT8 page.
+ */
+#ifndef BQ_H_
+#define BQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bq_status {
+    BQ_OK = 0,
+    BQ_ERR_INVALID_ARG = 1,     /* bad pointer, size, stride or dtype */
+    BQ_ERR_UNSUPPORTED = 2,     /* valid request no kernel implements */
+    BQ_ERR_ALIGNMENT = 3,       /* a forced kernel path needs aligned data */
+    BQ_ERR_WORKSPACE = 4,       /* workspace missing or too small */
+    BQ_ERR_CUDA = 5,            /* a CUDA runtime call failed */
+    BQ_ERR_DEVICE_TIMEOUT = 6   /* a bounded device-side wait gave up */
+} bq_status;
+
+typedef enum bq_dtype {
+    BQ_INT8 = 0,      /* int8 codes, Q = 127, int32 block partials */
+    BQ_FP8_E4M3 = 1   /* e4m3 codes, Q = 448, fp32 block partials */
+} bq_dtype;
+
+/* GEMM kernel families (for bq_set_path). */
+typedef enum bq_path {
+    BQ_PATH_AUTO = 0,     /* choose by shape and alignment */
+    BQ_PATH_SIMT = 1,     /* generic CUDA-core kernel: any shape/stride */
+    BQ_PATH_TCGEN05 = 2,  /* TMA + tcgen05 tensor-core kernel (large M) */
+    BQ_PATH_DECODE = 3    /* split-K weight-streaming kernel (small M) */
+} bq_path;
+
+/* ---- library information and errors ---------------------------------- */
+
+/* Library version, major*10000 + minor*100 + patch. */
+int bq_version(void);
+
+/* Static description of a status code (never NULL). */
+const char* bq_status_string(int status);
+
+/* Description of the last error raised on the calling host thread ("" if
+ * none).  The pointer stays valid until the next bq_* call on this thread. */
+const char* bq_last_error_message(void);
+
+/* Force the GEMM kernel family used by bq_gemm / bq_linear /
+ * bq_grouped_gemm on the calling host thread (BQ_PATH_AUTO restores the
+ * automatic choice).  A forced path that cannot run the given shape returns
+ * BQ_ERR_UNSUPPORTED or BQ_ERR_ALIGNMENT instead of falling back. */
+bq_status bq_set_path(int path);
+int bq_get_path(void);
+
+/* Read and clear the current device's status word, which kernels set when a
+ * bounded wait gives up (BQ_ERR_DEVICE_TIMEOUT, with the wait site in the
+ * message) or when they meet invalid device-side input such as an expert id
+ * out of range (BQ_ERR_INVALID_ARG).  Synchronises `stream`. */
+bq_status bq_check_device_status(void* stream);
+
+/* Self-test of the device status word: launches one tiny kernel that waits
+ * for a flag nothing sets, with an iteration limit of `spin_limit`; the wait
+ * runs out and records a timeout.  A following bq_check_device_status
+ * returns BQ_ERR_DEVICE_TIMEOUT.  Faults nothing and leaves the context
+ * usable. */
+bq_status bq_selftest_bounded_wait(int64_t spin_limit, void* stream);
+
+/* ---- configuration checks (host only) --------------------------------- */
+
+/* The three rejections of the block-wise INT8 config (page section 1):
+ * a block size requires an int8-serialised checkpoint
+ * (checkpoint_int8_serialized != 0), the block size has exactly two
+ * dimensions (n_block_dims == 2), and the activation scheme is dynamic
+ * (dynamic_activation != 0).  has_block_size == 0 accepts everything.
+ * Returns BQ_OK or BQ_ERR_INVALID_ARG with the reason in the message. */
+bq_status bq_check_block_config(int has_block_size, int checkpoint_int8_serialized,
+                                int64_t n_block_dims, int dynamic_activation);
+
+/* Tensor-parallel alignment of the block-wise INT8 page, section 3.
+ * Row-parallel (tp_size > 1 and input_size / input_size_per_partition ==
+ * tp_size): input_size_per_partition must be a multiple of block_k.
+ * Column-parallel: every output_partition_sizes[i] (host array of n_parts)
+ * must be a multiple of block_n.  Returns BQ_OK or BQ_ERR_INVALID_ARG. */
+bq_status bq_check_tp_partition(int64_t tp_size, int64_t input_size,
+                                int64_t input_size_per_partition,
+                                const int64_t* output_partition_sizes, int64_t n_parts,
+                                int64_t block_n, int64_t block_k);
+
+/* ---- dynamic activation quantisation ------------------------------ */
+
+/* x: bf16 [M, K], row stride ldx >= K.  Writes q [M, K] codes (row stride
+ * ldq >= K) and s: fp32 [ceil(K/group_k)][M] (K-block-major, dense).
+ * group_k >= 1; the last group of a row may be partial (ceil division) and
+ * takes its amax over its valid elements only.  dtype: bq_dtype.
+ * Block-wise INT8 page section 4 (dynamic, per token); groups of 1 x
+ * block_k so that each K-block has its own activation scale. */
+bq_status bq_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, int64_t group_k,
+                       int dtype, void* q, int64_t ldq, float* s, void* stream);
+
+/* ---- offline weight block quantisation ---------------------------- */
+
+/* w: fp32 [N, K] (row stride ldw >= K).  Writes q [N, K] (row stride
+ * ldq >= K) and s: fp32 [ceil(N/block_n)][ceil(K/block_k)] row-major, one
+ * scale per [block_n, block_k] block (amax over the block's valid elements
+ * / Q).  Block-wise INT8 page, structure diagram and section 2.  Not on the
+ * inference path: checkpoints arrive quantised. */
+bq_status bq_quant_weight(const float* w, int64_t N, int64_t K, int64_t ldw,
+                          int64_t block_n, int64_t block_k, int dtype, void* q,
+                          int64_t ldq, float* s, void* stream);
+
+/* ---- block-scaled GEMM ----------------------------------------- */
+
+/* Bytes of workspace bq_gemm needs for this problem (0 is possible). */
+bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_n,
+                                 int64_t block_k, int dtype, size_t* bytes);
+
+/* out[m, n] = bf16( sum_kb P_kb[m,n] * sa[kb*M + m] * sw[(n/block_n)*Kb + kb]
+ *                   + bias[n] )
+ * qa: codes [M, K] (row stride lda >= K); sa: fp32 [Kb][M] activation scales
+ *   from bq_quant_act with group_k == block_k;
+ * qw: codes [N, K] (row stride ldw >= K), sw: fp32 [ceil(N/block_n)][Kb];
+ * bias: bf16 [N] or NULL; out: bf16 [M, N] (row stride ldo >= N).
+ * block_k <= 65536 keeps INT8 block partials exact in int32.
+ * workspace: device memory of at least bq_gemm_workspace_size bytes (may be
+ *   NULL when that size is 0).  Its first use must see it zero-filled; every
+ *   successful call leaves it zero-filled again.  Calls sharing one
+ *   workspace must not overlap on the GPU.
+ * Block-wise INT8 page sections 2 and 4 (apply_w8a8_block_int8_linear with
+ * input_scale=None, after the activation quantisation); blockwise FP8 of the
+ * SGLang quantization doc. */
+bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, int64_t ldw,
+                  const float* sw, int64_t M, int64_t N, int64_t K, int64_t block_n,
+                  int64_t block_k, int dtype, const void* bias, void* out, int64_t ldo,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace for bq_linear: the activation codes and scales plus bq_gemm's. */
+bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_n,
+                                   int64_t block_k, int dtype, size_t* bytes);
+
+/* The whole linear layer: bq_quant_act(x, group_k = block_k) then bq_gemm,
+ * i.e. apply_w8a8_block_int8_linear(input, weight, block_size, weight_scale,
+ * input_scale=None, bias) of the block-wise INT8 page, section 4.
+ * x: bf16 [M, K] (row stride ldx >= K); other arguments as bq_gemm.  The
+ * workspace (bq_linear_workspace_size bytes) follows bq_gemm's rules. */
+bq_status bq_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void* qw,
+                    int64_t ldw, const float* sw, int64_t N, int64_t block_n, int64_t block_k,
+                    int dtype, const void* bias, void* out, int64_t ldo, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* ---- MoE (block-wise INT8 page, sections 5 and 6) ---------------- */
+
+/* Bytes of workspace bq_moe_permute needs. */
+bq_status bq_moe_permute_workspace_size(int64_t T, int64_t topk, int64_t E, size_t* bytes);
+
+/* Group the T*topk (token, slot) pairs by expert, stably (by expert, then by
+ * flat index t*topk + j).  topk_ids: int32 [T, topk], each in [0, E).
+ * Writes expert_offsets: int32 [E+1] (exclusive prefix of per-expert counts,
+ * expert_offsets[E] = T*topk), perm: int32 [T*topk] (flat pair index at
+ * each permuted row) and inv_perm: int32 [T*topk] (permuted row of each
+ * pair).  An id outside [0, E) is placed nowhere (expert_offsets[E] then
+ * falls short of T*topk) and is recorded in the device status word, which
+ * bq_check_device_status reports as BQ_ERR_INVALID_ARG.  Group sizes stay
+ * on the device (no host read-back). */
+bq_status bq_moe_permute(const int32_t* topk_ids, int64_t T, int64_t topk, int64_t E,
+                         int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Activation quantisation of the routed rows: permuted row r holds token
+ * perm[r] / topk.  x: bf16 [T, H] (row stride ldx >= H).  Writes q
+ * [T*topk, H] (row stride ldq >= H) and s fp32 [ceil(H/group_k)][T*topk].
+ * Codes are identical to bq_quant_act of x followed by a row gather. */
+bq_status bq_moe_quant_gather(const void* x, int64_t T, int64_t H, int64_t ldx,
+                              const int32_t* perm, int64_t topk, int64_t group_k, int dtype,
+                              void* q, int64_t ldq, float* s, void* stream);
+
+/* Bytes of workspace bq_grouped_gemm needs. */
+bq_status bq_grouped_gemm_workspace_size(int64_t R, int64_t N, int64_t K, int64_t E,
+                                         int64_t block_n, int64_t block_k, int dtype,
+                                         size_t* bytes);
+
+/* Per expert e, rows [expert_offsets[e], expert_offsets[e+1]) of qa run the
+ * block-scaled GEMM against expert e's weight:
+ * qa: codes [R, K] (row stride lda), sa: fp32 [Kb][R];
+ * expert_offsets: DEVICE int32 [E+1], nondecreasing, offsets[0] = 0,
+ *   offsets[E] <= R (rows past offsets[E] are left untouched);
+ * qw: codes [E, N, K] (dense), sw: fp32 [E][Nbs][Kb] with Nbs weight-scale
+ *   rows per expert;
+ * n_seam: 0 for a plain weight (Nbs = ceil(N/block_n)); for a fused gate+up
+ *   weight the gate/up boundary I (= N/2): rows [0, I) use scale row n/bn and
+ *   rows [I, N) use ceil(I/bn) + (n-I)/bn, so Nbs = 2*ceil(I/bn)
+ *   (block-wise INT8 page, section 5);
+ * out: bf16 [R, N] (row stride ldo >= N). */
+bq_status bq_grouped_gemm(const void* qa, int64_t lda, const float* sa, int64_t R,
+                          const int32_t* expert_offsets, int64_t E, const void* qw,
+                          const float* sw, int64_t N, int64_t K, int64_t block_n,
+                          int64_t block_k, int64_t n_seam, int dtype, void* out, int64_t ldo,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* h = bf16(silu(y[r, i]) * y[r, I + i]) (gate then up, block-wise INT8
+ * page section 5 "gate + up fused"; SiLU is the reading for a gate/up pair),
+ * then the activation quantisation of h with 1 x group_k groups.
+ * y: bf16 [R, 2I] (row stride ldy >= 2I).  Writes q [R, I] (row stride
+ * ldq >= I), s fp32 [ceil(I/group_k)][R] and, if h_out is not NULL, h as
+ * bf16 [R, I] (dense). */
+bq_status bq_moe_silu_mul_quant(const void* y, int64_t ldy, int64_t R, int64_t I,
+                                int64_t group_k, int dtype, void* q, int64_t ldq, float* s,
+                                void* h_out, void* stream);
+
+/* out[t, n] = bf16( sum_j topk_w[t*topk + j] * y[inv_perm[t*topk + j], n] ),
+ * fp32 accumulation, one rounding.  y: bf16 [T*topk, H] (row stride ldy),
+ * topk_w: fp32 [T, topk], out: bf16 [T, H] (row stride ldo). */
+bq_status bq_moe_combine(const void* y, int64_t ldy, const int32_t* inv_perm,
+                         const float* topk_w, int64_t T, int64_t topk, int64_t H, void* out,
+                         int64_t ldo, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H_ */

@@ -158,7 +158,7 @@ def code_values(q: np.ndarray, dtype: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# a1 / a2: quantisation
+# quantisation
 # --------------------------------------------------------------------------
 
 def quant_act(x_bf16: np.ndarray, group_k: int, dtype: int):
@@ -199,7 +199,7 @@ def quant_weight_gate_up(w13: np.ndarray, I: int, bn: int, bk: int, dtype: int):
 
 
 # --------------------------------------------------------------------------
-# a3 / a4: GEMM
+# GEMM
 # --------------------------------------------------------------------------
 
 def gemm(qa, sa, qw, sw, bn: int, bk: int, dtype: int, bias_bf16=None, seam: int = 0):
@@ -244,7 +244,7 @@ def dequant_dot(qa, sa, qw, sw, bn: int, bk: int, dtype: int, m: int, n: int,
 
 
 # --------------------------------------------------------------------------
-# a5-a9: MoE
+# MoE
 # --------------------------------------------------------------------------
 
 def moe_permute(ids: np.ndarray, E: int):

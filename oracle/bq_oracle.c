@@ -173,7 +173,7 @@ static double code_value(uint8_t c, int dtype) {
 }
 
 /* ------------------------------------------------------------------------ */
-/* a1: dynamic activation quantisation, groups 1 x group_k ([BWI8] §4)       */
+/* dynamic activation quantisation, groups 1 x group_k ([BWI8] §4)       */
 /* ------------------------------------------------------------------------ */
 
 /* x: bf16 [M, K] (row stride ldx); q: [M, K] bytes (row stride ldq);
@@ -196,7 +196,7 @@ void bq_ref_quant_act(const uint16_t* x, long M, long K, long ldx, long group_k,
 }
 
 /* ------------------------------------------------------------------------ */
-/* a2: offline weight block quantisation ([BWI8] §2, structure diagram)     */
+/* offline weight block quantisation ([BWI8] §2, structure diagram)     */
 /* ------------------------------------------------------------------------ */
 
 /* w: fp32 [N, K] row-major (stride ldw); q: [N, K] bytes (stride ldq);
@@ -224,7 +224,7 @@ void bq_ref_quant_weight(const float* w, long N, long K, long ldw, long bn, long
 }
 
 /* ------------------------------------------------------------------------ */
-/* a3/a4: block-scaled GEMM ([BWI8] §2, §4; [QDOC] blockwise FP8)            */
+/* block-scaled GEMM ([BWI8] §2, §4; [QDOC] blockwise FP8)            */
 /* ------------------------------------------------------------------------ */
 
 /* Weight-scale row of output column n.  With seam == 0 (or >= N) this is
@@ -296,7 +296,7 @@ double bq_ref_dequant_dot(const uint8_t* qa, long lda, const float* sa, const ui
 }
 
 /* ------------------------------------------------------------------------ */
-/* a5: MoE token permutation ([BWI8] §5-§6: per-expert weights, routed      */
+/* MoE token permutation ([BWI8] §5-§6: per-expert weights, routed      */
 /* tokens).  Stable order: by expert, then by flat slot index t*topk + j.   */
 /* ------------------------------------------------------------------------ */
 
@@ -324,7 +324,7 @@ int bq_ref_moe_permute(const int32_t* ids, long T, long topk, long E, int32_t* o
     return 0;
 }
 
-/* a7: h = silu(g) * u rounded once to bf16, g = y[r, i], u = y[r, I + i]
+/* h = silu(g) * u rounded once to bf16, g = y[r, i], u = y[r, I + i]
  * ("gate + up fused", [BWI8] §5; SiLU is the reading for a gate/up pair).
  * silu(g) = g / (1 + exp(-g)), in fp64. */
 void bq_ref_silu_mul(const uint16_t* y, long R, long I, long ldy, uint16_t* h) {
@@ -338,7 +338,7 @@ void bq_ref_silu_mul(const uint16_t* y, long R, long I, long ldy, uint16_t* h) {
     }
 }
 
-/* a9: out[t, n] = bf16( sum_j w[t, j] * y[inv_perm[t*topk + j], n] ), fp64. */
+/* out[t, n] = bf16( sum_j w[t, j] * y[inv_perm[t*topk + j], n] ), fp64. */
 void bq_ref_moe_combine(const uint16_t* y, long ldy, const int32_t* inv_perm,
                         const float* w, long T, long topk, long H, uint16_t* out) {
     for (long t = 0; t < T; t++) {

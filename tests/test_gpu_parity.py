@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Quantised codes and scales must match bit for bit; GEMM outputs must meet
+max|d| <= 1e-2 max|ref| and relative Frobenius <= 2e-3 against the fp64
+oracle on the same codes, and lie within one bf16 ulp of the exact value.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_w8a8_b200 as bq
+import bq_synth
+import oracle
+from gpu_util import (assert_codes_equal, assert_gemm_close, assert_scales_equal, bf16_ulp,
+                      bf16_values, dev_bf16, dev_f32, dev_i32, dev_u8, host_bits)
+
+pytestmark = pytest.mark.gpu
+
+INT8, FP8 = bq.INT8, bq.FP8_E4M3
+
+
+@pytest.fixture(autouse=True)
+def _reset_path():
+    bq.set_path(bq.PATH_AUTO)
+    yield
+    bq.set_path(bq.PATH_AUTO)
+    bq.check_device_status()
+
+
+def act_bits(M, K, seed, n_out=0, scale=1.0):
+    return host_bits(bq_synth.activations(M, K, seed, n_out, scale))
+
+
+# --------------------------------------------------------------------------
+# activation quantisation: bit-exact
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,K,gk,pad", [
+    (16, 200, 128, 0),      # tiny workload: partial second group
+    (64, 4096, 128, 0),     # decode width
+    (37, 1000, 128, 8),     # ragged K, padded row stride
+    (5, 300, 32, 0),
+    (3, 700, 256, 0),       # group longer than 128 (two-pass)
+    (7, 333, 100, 3),       # group not a multiple of 4 (scalar path)
+    (1, 1, 128, 0),
+])
+def test_quant_act_bit_exact(dtype, M, K, gk, pad):
+    xb = act_bits(M, K + pad, 11 + M, max(1, (K + pad) // 100), 30.0)
+    xb[0, :] = 0                                   # an all-zero row
+    if M > 2:
+        xb[2, :] = 0x0001                          # subnormal amax: scale underflows to 0
+    x = dev_bf16(xb)[:, :K]
+    q, s = bq.quant_act(x, gk, dtype)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.quant_act(np.ascontiguousarray(xb[:, :K]), gk, dtype)
+    assert_codes_equal(q, q_ref, "codes")
+    assert_scales_equal(s, s_ref, "scales")
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+def test_quant_act_extremes(dtype):
+    # large, tiny and tie-making values in one group
+    vals = np.array([3.0e38, -1.0e-38, 2.5, -2.5, 0.5, 1e-40, -0.0, 448.0] * 16, np.float32)
+    xb = host_bits(torch.from_numpy(vals).to(torch.bfloat16))[None, :]
+    ties = np.concatenate([[127.0], np.arange(-20, 20) + 0.5, np.zeros(87)])
+    tb = host_bits(torch.from_numpy(ties.astype(np.float32)).to(torch.bfloat16))[None, :]
+    xb = np.concatenate([xb, tb], 0)
+    q, s = bq.quant_act(dev_bf16(xb), 128, dtype)
+    q_ref, s_ref = oracle.quant_act(xb, 128, dtype)
+    assert_codes_equal(q, q_ref, "codes")
+    assert_scales_equal(s, s_ref, "scales")
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("N,K,bn,bk", [(320, 200, 128, 128), (256, 384, 128, 128),
+                                       (100, 77, 32, 16)])
+def test_quant_weight_bit_exact(dtype, N, K, bn, bk):
+    w = bq_synth.weights(N, K, 0.02, 3)
+    w[0, :5] = 0.0
+    q, s = bq.quant_weight(w.cuda(), bn, bk, dtype)
+    q_ref, s_ref = oracle.quant_weight(w.numpy(), bn, bk, dtype)
+    assert_codes_equal(q, q_ref, "weight codes")
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# block-scaled GEMM
+# --------------------------------------------------------------------------
+
+def make_problem(M, N, K, bn, bk, dtype, seed, bias=False, n_out=3):
+    """Operands quantised by the ORACLE (codes and scales are its outputs)."""
+    xb = act_bits(M, K, seed, n_out, 20.0)
+    w = bq_synth.weights(N, K, 0.02, seed).numpy()
+    qa, sa = oracle.quant_act(xb, bk, dtype)
+    qw, sw = oracle.quant_weight(w, bn, bk, dtype)
+    bb = host_bits(torch.randn(N, generator=torch.Generator().manual_seed(seed)).to(
+        torch.bfloat16)) if bias else None
+    return xb, qa, sa, qw, sw, bb
+
+
+GEMM_SHAPES = [
+    # M, N, K, bn, bk
+    (16, 320, 200, 128, 128),   # the tiny workload: 3x2 scale grid, partial blocks
+    (300, 520, 1000, 128, 128), # several tiles, ragged M, N, K
+    (1, 256, 512, 128, 128),
+    (129, 257, 384, 64, 128),
+    (40, 96, 250, 96, 64),      # odd block sizes
+]
+
+
+@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_AUTO])
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,N,K,bn,bk", GEMM_SHAPES)
+def test_gemm_vs_oracle(path, dtype, M, N, K, bn, bk):
+    _, qa, sa, qw, sw, bb = make_problem(M, N, K, bn, bk, dtype, 100 + M, bias=(M % 2 == 0))
+    bq.set_path(path)
+    out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), bn, bk, dtype,
+                  bias=None if bb is None else dev_bf16(bb))
+    torch.cuda.synchronize()
+    ref = oracle.gemm(qa, sa, qw, sw, bn, bk, dtype, bias_bf16=bb)
+    assert_gemm_close(out, ref, f"gemm path={path} dtype={dtype} {M}x{N}x{K}")
+
+
+def test_gemm_strided_operands_and_output():
+    M, N, K, bn, bk = 70, 200, 300, 128, 128
+    _, qa, sa, qw, sw, _ = make_problem(M, N, K, bn, bk, INT8, 7)
+    qa_pad = np.zeros((M, K + 20), np.uint8)
+    qa_pad[:, :K] = qa
+    qw_pad = np.zeros((N, K + 12), np.uint8)
+    qw_pad[:, :K] = qw
+    big = torch.full((M, N + 10), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = big[:, 3:3 + N]
+    bq.gemm(dev_u8(qa_pad)[:, :K], dev_f32(sa.T), dev_u8(qw_pad)[:, :K], dev_f32(sw), bn, bk,
+            INT8, out=out)
+    torch.cuda.synchronize()
+    assert_gemm_close(out, oracle.gemm(qa, sa, qw, sw, bn, bk, INT8), "strided")
+    assert torch.isnan(big[:, :3]).all() and torch.isnan(big[:, 3 + N:]).all()
+
+
+def test_gemm_k_zero_gives_bias():
+    M, N = 3, 5
+    bias = torch.randn(N).to(torch.bfloat16).cuda()
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    qa = torch.zeros(M, 0, dtype=torch.uint8, device="cuda")
+    qw = torch.zeros(N, 0, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(0, M, device="cuda")
+    bq.gemm(qa, s, qw, torch.zeros(1, 0, device="cuda"), 128, 128, INT8, bias=bias, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, bias[None, :].expand(M, N))
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+def test_linear_tiny_workload(dtype):
+    cfg = bq_synth.TINY
+    a, w = bq_synth.linear_inputs(cfg)
+    xb = host_bits(a)
+    qw_ref, sw_ref = oracle.quant_weight(w.numpy(), 128, 128, dtype)
+    out = bq.linear(dev_bf16(xb), dev_u8(qw_ref), dev_f32(sw_ref), 128, 128, dtype)
+    torch.cuda.synchronize()
+    qa, sa = oracle.quant_act(xb, 128, dtype)
+    assert sw_ref.shape == (3, 2)
+    assert_gemm_close(out, oracle.gemm(qa, sa, qw_ref, sw_ref, 128, 128, dtype), "linear")
+
+
+# --------------------------------------------------------------------------
+# MoE steps
+# --------------------------------------------------------------------------
+
+def moe_problem(T=200, H=256, I=192, E=8, topk=2, seed=21, dtype=INT8):
+    x = act_bits(T, H, seed)
+    ids, tw = bq_synth.routing(T, E, topk, seed)
+    w13 = bq_synth.weights(2 * I, H, 0.02, seed, batch=E).numpy()
+    w2 = bq_synth.weights(H, I, 0.02, seed + 1, batch=E).numpy()
+    q13, s13 = zip(*[oracle.quant_weight_gate_up(w13[e], I, 128, 128, dtype) for e in range(E)])
+    q2, s2 = zip(*[oracle.quant_weight(w2[e], 128, 128, dtype) for e in range(E)])
+    return dict(x=x, ids=ids, tw=tw, q13=np.stack(q13), s13=np.stack(s13), q2=np.stack(q2),
+                s2=np.stack(s2), T=T, H=H, I=I, E=E, topk=topk, dtype=dtype)
+
+
+def test_moe_permute_bit_exact():
+    for T, E, topk in [(200, 8, 2), (1000, 8, 2), (37, 5, 3), (4096, 8, 2)]:
+        ids, _ = bq_synth.routing(T, E, topk, T)
+        off, perm, inv = bq.moe_permute(dev_i32(ids), E)
+        o_ref, p_ref, i_ref = oracle.moe_permute(ids, E)
+        assert np.array_equal(off.cpu().numpy(), o_ref)
+        assert np.array_equal(perm.cpu().numpy(), p_ref)
+        assert np.array_equal(inv.cpu().numpy(), i_ref)
+
+
+def test_moe_permute_skewed_and_empty_experts():
+    ids = np.zeros((3000, 2), np.int32)
+    ids[:, 1] = 7
+    ids[::7, 0] = 3
+    off, perm, inv = bq.moe_permute(dev_i32(ids), 8)
+    o_ref, p_ref, i_ref = oracle.moe_permute(ids, 8)
+    assert np.array_equal(off.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy(), p_ref)
+
+
+def test_moe_layer_stages_vs_oracle():
+    p = moe_problem()
+    T, H, I, E, topk, dt = p["T"], p["H"], p["I"], p["E"], p["topk"], p["dtype"]
+    x = dev_bf16(p["x"])
+    off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), E)
+    o_ref, p_ref, i_ref = oracle.moe_permute(p["ids"], E)
+    # quant + gather: identical to quantising then gathering rows
+    qa, sa = bq.moe_quant_gather(x, perm, topk, 128, dt)
+    qx_ref, sx_ref = oracle.quant_act(p["x"], 128, dt)
+    rows = p_ref // topk
+    assert_codes_equal(qa, qx_ref[rows], "gathered codes")
+    assert_scales_equal(sa, np.ascontiguousarray(sx_ref[rows]), "gathered scales")
+    # w13 grouped GEMM with the gate/up seam (I = 192 is not a multiple of 128)
+    y13 = bq.grouped_gemm(qa, sa, off, dev_u8(p["q13"]), dev_f32(p["s13"]), 128, 128,
+                          n_seam=I, dtype=dt)
+    torch.cuda.synchronize()
+    ref13 = oracle.grouped_gemm(qx_ref[rows], sx_ref[rows], o_ref, p["q13"], p["s13"], 128,
+                                128, dt, seam=I)
+    assert_gemm_close(y13, ref13, "w13")
+    # silu * up, requantised: h within one bf16 ulp, codes exact for the GPU's h
+    q2a, s2a, h = bq.moe_silu_mul_quant(y13, I, 128, dt, want_h=True)
+    torch.cuda.synchronize()
+    y13_bits = host_bits(y13)
+    h_ref = oracle.bf16_to_f64(oracle.silu_mul(y13_bits, I))
+    hv = bf16_values(h)
+    assert (np.abs(hv - h_ref) <= bf16_ulp(np.maximum(np.abs(hv), np.abs(h_ref)))).all()
+    qh_ref, sh_ref = oracle.quant_act(host_bits(h), 128, dt)
+    assert_codes_equal(q2a, qh_ref, "requantised codes")
+    assert_scales_equal(s2a, sh_ref, "requantised scales")
+    # w2 grouped GEMM
+    y2 = bq.grouped_gemm(q2a, s2a, off, dev_u8(p["q2"]), dev_f32(p["s2"]), 128, 128, 0, dt)
+    torch.cuda.synchronize()
+    ref2 = oracle.grouped_gemm(qh_ref, sh_ref, o_ref, p["q2"], p["s2"], 128, 128, dt)
+    assert_gemm_close(y2, ref2, "w2")
+    # combine: fp32 accumulate, one rounding
+    out = bq.moe_combine(y2, inv, dev_f32(p["tw"]))
+    torch.cuda.synchronize()
+    comb_ref = oracle.bf16_to_f64(oracle.moe_combine(host_bits(y2), i_ref, p["tw"]))
+    ov = bf16_values(out)
+    assert (np.abs(ov - comb_ref) <= bf16_ulp(np.maximum(np.abs(ov), np.abs(comb_ref)))).all()
+
+
+def test_grouped_gemm_leaves_rows_past_offsets_untouched():
+    p = moe_problem(T=50, H=128, I=128, E=4)
+    off = np.array([0, 10, 10, 30, 60], np.int32)     # 60 of the 100 rows routed
+    R = 100
+    qa = np.random.default_rng(0).integers(-100, 100, (R, 128)).astype(np.int8).view(np.uint8)
+    sa = np.full((R, 1), 0.01, np.float32)
+    out = torch.full((R, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    bq.grouped_gemm(dev_u8(qa), dev_f32(sa.T), dev_i32(off), dev_u8(p["q2"][:4]),
+                    dev_f32(p["s2"][:4]), 128, 128, 0, INT8, out=out)
+    torch.cuda.synchronize()
+    ref = oracle.grouped_gemm(qa[:60], sa[:60], off, p["q2"][:4], p["s2"][:4], 128, 128, INT8)
+    assert_gemm_close(out[:60], ref, "grouped")
+    assert (out[60:] == 7.0).all()
+
+
+# --------------------------------------------------------------------------
+# device status word
+# --------------------------------------------------------------------------
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    bq.selftest_bounded_wait(2000)
+    with pytest.raises(bq.BqError) as ei:
+        bq.check_device_status()
+    assert ei.value.status == bq.ERR_DEVICE_TIMEOUT
+    bq.check_device_status()          # cleared
+    q, s = bq.quant_act(torch.ones(2, 128, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert (q.cpu().numpy().view(np.int8) == 127).all()
+
+
+def test_bad_expert_id_is_reported():
+    ids = np.array([[0, 1], [9, 2], [3, -1]], np.int32)
+    off, perm, inv = bq.moe_permute(dev_i32(ids), 8)
+    with pytest.raises(bq.BqError) as ei:
+        bq.check_device_status()
+    assert ei.value.status == bq.ERR_INVALID_ARG
+    assert off.cpu().numpy()[-1] == 4      # the two bad pairs are placed nowhere

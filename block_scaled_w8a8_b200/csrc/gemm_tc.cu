@@ -1,0 +1,438 @@
+// gemm_tc.cu -- block-scaled GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// out[m, n] = bf16( sum_kb P_kb[m, n] * sa[kb][m] * sw[nb(n)][kb] + bias[n] )
+// (block-wise INT8 page, sections 2 and 4; blockwise FP8 of the SGLang
+// quantization doc, "GEMM backends for FP4/FP8"), for block_n = block_k = 128.
+//
+// Design (persistent, warp-specialised, one CTA per SM):
+//   warp 0      TMA producer: per K-block, one 128x128 A tile and one BNx128
+//               W tile (K-major, 128-byte swizzle) into an S-stage ring.
+//   warp 1      MMA issuer (lane 0): 4 x tcgen05.mma (K = 32 each) per K-block
+//               into a TMEM buffer; the buffer holds exactly one K-block's
+//               partial P_kb (int32 for kind::i8, fp32 for kind::f8f6f4).
+//               Two TMEM buffers alternate so the MMA of block kb+1 overlaps
+//               the promotion of block kb.  Also owns the TMEM allocation.
+//   warps 4-7   epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
+//               per thread), promotes acc += P_kb * (sa[kb][m] * sw[nb][kb])
+//               in fp32 registers, frees the buffer, and after the last
+//               K-block adds the bias and stores bf16.
+// A tile scheduler walks (expert, m-block, n-block) tiles; a dense problem is
+// one expert.  The grouped (MoE) problem reads its expert row ranges from
+// device memory, so no host read-back is needed.  Rows of a tile past the
+// expert's range are computed but never stored.
+//
+// Every mbarrier wait is bounded (2 s); on expiry the CTA records a timeout
+// in the device status word, drains its in-flight TMA loads and MMAs, frees
+// its tensor memory and exits.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <mutex>
+
+#include "bq_common.cuh"
+#include "bq_internal.h"
+#include "gemm_tc.h"
+#include "sm100.cuh"
+
+namespace bq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BK = 128;
+constexpr int kThreads = 256;        // 8 warps: producer, MMA, 2 idle, 4 epilogue
+constexpr int kMaxE = 256;
+
+struct TcParams {
+  const float* sa; int64_t sa_rows;
+  const float* sw; int64_t sw_expert_stride;
+  int64_t M, N, K, Kb, seam;
+  const int32_t* offsets; int E;
+  const uint16_t* bias;
+  uint16_t* out; int64_t ldo;
+  int nblk;
+  unsigned* status;
+};
+
+template <int BN, int S>
+struct Smem {
+  static constexpr uint32_t kA = BM * BK, kB = BN * BK;
+  static constexpr uint32_t kStages = S * (kA + kB);
+  static constexpr uint32_t kBars = (2 * S + 4 + 2) * 8;
+  static constexpr uint32_t kMisc = 8 + 2 * (kMaxE + 1) * 4;
+  static constexpr uint32_t kTotal = 1024 + kStages + kBars + kMisc;
+};
+
+__device__ __forceinline__ int64_t wrow_block(int64_t n, int64_t seam, int64_t N) {
+  if (seam <= 0 || seam >= N || n < seam) return n >> 7;
+  return ((seam + 127) >> 7) + ((n - seam) >> 7);
+}
+
+// Tile t -> (expert, m-block, n-block); m-blocks vary fastest so concurrent
+// CTAs share W tiles and the A operand of an expert stays in L2.
+__device__ __forceinline__ void decode_tile(int t, const int* tp, const int* off, int E, int nblk,
+                                            int& e_hint, int& e, int& mb, int& nb) {
+  int ee = e_hint;
+  while (ee + 1 < E && t >= tp[ee + 1]) ++ee;
+  e_hint = ee;
+  e = ee;
+  const int local = t - tp[ee];
+  const int mblocks = (off[ee + 1] - off[ee] + BM - 1) / BM;
+  mb = local % mblocks;
+  nb = local / mblocks;
+}
+
+template <int DT>
+__device__ __forceinline__ float partial_to_float(uint32_t bits) {
+  if constexpr (DT == kInt8) return __int2float_rn((int)bits);
+  else return __uint_as_float(bits);
+}
+
+template <int DT, int BN, int S>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcParams p) {
+  using L = Smem<BN, S>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * L::kA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStages);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 6);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* off_s = reinterpret_cast<int*>(tmem_slot + 2);
+  int* tp_s = off_s + (kMaxE + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 4);
+    }
+    mbar_init(smem_u32(&drain[0]), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  // expert row ranges (sanitised: clamped to [0, M] and nondecreasing)
+  if (threadIdx.x == 32) {
+    int prev = 0;
+    bool bad = false;
+    for (int e = 0; e <= E; ++e) {
+      int v = p.offsets ? p.offsets[e] : (e == 0 ? 0 : (int)p.M);
+      if (e == 0 && v != 0) bad = true;
+      int c = min(max(v, prev), (int)p.M);
+      if (c != v) bad = true;
+      off_s[e] = (e == 0) ? 0 : c;
+      prev = off_s[e];
+    }
+    if (bad) record_status(p.status, kStatusBadInput, 0x201u);
+    tp_s[0] = 0;
+    for (int e = 0; e < E; ++e)
+      tp_s[e + 1] = tp_s[e] + ((off_s[e + 1] - off_s[e] + BM - 1) / BM) * p.nblk;
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 2 * BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = tp_s[E];
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued_parity[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) issued_parity[s] = -1;
+    int e_hint = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      int e, mb, nb;
+      decode_tile(t, tp_s, off_s, E, p.nblk, e_hint, e, mb, nb);
+      const int a_row = off_s[e] + mb * BM;
+      const int b_row = e * (int)p.N + nb * BN;
+      for (int kb = 0; kb < p.Kb; ++kb) {
+        if (!warp_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.status, 0x301u)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kA + L::kB);
+          tma_load_2d(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, smem_u32(&full[stage]));
+          tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, b_row, smem_u32(&full[stage]));
+        }
+        issued_parity[stage] = (int)phase;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      // drain: wait (bounded) for every load this warp issued
+      for (int s = 0; s < S; ++s) {
+        if (issued_parity[s] < 0) continue;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(&full[s]), (uint32_t)issued_parity[s]) &&
+               globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t idesc = instr_desc<DT>(BM, BN);
+    int stage = 0;
+    uint32_t phase = 0, kcount = 0;
+    int e_hint = 0;
+    bool ok = true, issued_any = false;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int kb = 0; kb < p.Kb; ++kb) {
+        const uint32_t buf = kcount & 1, tround = kcount >> 1;
+        if (!warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag, p.status, 0x302u) ||
+            !warp_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x303u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t d = tmem_base + buf * BN;
+          const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * L::kA));
+          const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * L::kB));
+#pragma unroll
+          for (int j = 0; j < BK / 32; ++j)
+            mma<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+          mma_commit(smem_u32(&empty[stage]));
+          mma_commit(smem_u32(&tfull[buf]));
+        }
+        __syncwarp();
+        issued_any = true;
+        ++kcount;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    (void)e_hint;
+    if (!ok && issued_any) {
+      if (lane == 0) mma_commit(smem_u32(&drain[0]));
+      __syncwarp();
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(smem_u32(&drain[0]), 0) && globaltimer() - t0 < 100000000ull) {
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------- epilogue ----------------
+    const int q = warp & 3;
+    const int rit = 32 * q + lane;                 // row inside the tile
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    uint32_t kcount = 0;
+    int e_hint = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      int e, mb, nb;
+      decode_tile(t, tp_s, off_s, E, p.nblk, e_hint, e, mb, nb);
+      const int row0 = off_s[e] + mb * BM;
+      const int64_t m = (int64_t)row0 + rit;
+      const bool row_ok = rit < off_s[e + 1] - row0;
+      const int64_t n0 = (int64_t)nb * BN;
+      const float* sw_e = p.sw + (int64_t)e * p.sw_expert_stride;
+      float acc[BN];
+#pragma unroll
+      for (int i = 0; i < BN; ++i) acc[i] = 0.f;
+      float sa_next = row_ok ? p.sa[m] : 0.f;     // K-block 0
+      for (int kb = 0; kb < p.Kb; ++kb) {
+        const uint32_t buf = kcount & 1, tround = kcount >> 1;
+        const float sa_v = sa_next;
+        if (kb + 1 < p.Kb) sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
+        if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x304u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          const int64_t nc = n0 + 32 * c;
+          const float swv = nc < p.N ? __ldg(sw_e + wrow_block(nc, p.seam, p.N) * p.Kb + kb) : 0.f;
+          const float f = sa_v * swv;
+          uint32_t r[32];
+          tmem_ld32(tmem_base + lane_base + buf * BN + 32 * c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            acc[32 * c + i] = fmaf(partial_to_float<DT>(r[i]), f, acc[32 * c + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+        ++kcount;
+      }
+      if (!ok) break;
+      if (row_ok) {
+        uint16_t* orow = p.out + m * p.ldo + n0;
+        const bool full_n = n0 + BN <= p.N;
+        const bool vec = full_n && ((reinterpret_cast<uintptr_t>(orow) & 15) == 0);
+        if (vec) {
+#pragma unroll
+          for (int j = 0; j < BN; j += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              float v0 = acc[j + 2 * h], v1 = acc[j + 2 * h + 1];
+              if (p.bias) {
+                v0 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h));
+                v1 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h + 1));
+              }
+              w[h] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
+            }
+            *reinterpret_cast<uint4*>(orow + j) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            if (n0 + j < p.N) {
+              float v = acc[j];
+              if (p.bias) v += bf16_bits_to_float(__ldg(p.bias + n0 + j));
+              orow[j] = float_to_bf16_bits(v);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+// ---- host side ------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// Row-major [rows, inner] uint8 tensor with row stride ld_bytes; box
+// [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes,
+               uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {ld_bytes};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (n[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
+  }
+  return n[dev];
+}
+
+template <int DT, int BN, int S>
+cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
+  using L = Smem<BN, S>;
+  auto kern = gemm_tc_kernel<DT, BN, S>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::kTotal);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tA, tB;
+  if (!make_tmap(&tA, a.qa, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.lda, BM) ||
+      !make_tmap(&tB, a.qw, (uint64_t)a.K, (uint64_t)(a.N * a.E), (uint64_t)a.ldw, BN))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.sa = a.sa; p.sa_rows = a.sa_rows;
+  p.sw = a.sw; p.sw_expert_stride = a.sw_expert_stride;
+  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK; p.seam = a.seam;
+  p.offsets = a.offsets; p.E = (int)a.E;
+  p.bias = static_cast<const uint16_t*>(a.bias);
+  p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;
+  p.nblk = (int)((a.N + BN - 1) / BN);
+  p.status = a.status;
+  const int64_t mblk_bound = (a.M + BM - 1) / BM + (a.offsets ? a.E : 0);
+  const int64_t tiles_bound = mblk_bound * p.nblk;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles_bound, sm_count()));
+  kern<<<grid, kThreads, L::kTotal, st>>>(tA, tB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(const GemmArgs& a, char* why, size_t n) {
+  auto no = [&](const char* msg) {
+    if (why) snprintf(why, n, "tcgen05 path: %s", msg);
+    return false;
+  };
+  if (a.bn != 128 || a.bk != 128) return no("needs block_n = block_k = 128");
+  if (a.K < 1) return no("needs K >= 1");
+  if (a.lda % 16 != 0 || a.ldw % 16 != 0) return no("row strides must be multiples of 16 bytes");
+  if ((reinterpret_cast<uintptr_t>(a.qa) & 15) || (reinterpret_cast<uintptr_t>(a.qw) & 15))
+    return no("operands must be 16-byte aligned");
+  if (a.seam % 128 != 0) return no("the gate/up seam must be a multiple of 128");
+  if (a.E > kMaxE) return no("at most 256 experts");
+  if (a.M > INT32_MAX || a.N * a.E > INT32_MAX || a.K > INT32_MAX) return no("sizes exceed int32");
+  if (!encode_fn()) return no("cuTensorMapEncodeTiled is unavailable");
+  return true;
+}
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
+  if (a.M == 0 || a.N == 0) return cudaSuccess;
+  if (a.dtype == kInt8) return launch_typed<kInt8, 128, 6>(a, st);
+  return launch_typed<kFp8, 128, 6>(a, st);
+}
+
+}  // namespace bq

@@ -1,0 +1,15 @@
+// gemm_tc.h -- the tcgen05 tensor-core GEMM (dense and grouped).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "bq_internal.h"
+
+namespace bq {
+
+// True if the tensor-core kernel can run this problem; otherwise writes why.
+bool tc_supported(const GemmArgs& a, char* why, size_t n);
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
+
+}  // namespace bq

@@ -122,6 +122,42 @@ def test_gemm_vs_oracle(path, dtype, M, N, K, bn, bk):
     assert_gemm_close(out, ref, f"gemm path={path} dtype={dtype} {M}x{N}x{K}")
 
 
+TC_SHAPES = [
+    # M, N, K: block 128x128, K a multiple of 16 bytes (TMA row stride)
+    (128, 128, 128),
+    (300, 520, 1008),     # ragged M and N tiles, partial last K-block (112)
+    (1, 256, 512),
+    (257, 640, 2048),
+    (64, 1280, 384),
+    (1000, 384, 4096),
+]
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,N,K", TC_SHAPES)
+def test_gemm_tcgen05_vs_oracle(dtype, M, N, K):
+    _, qa, sa, qw, sw, bb = make_problem(M, N, K, 128, 128, dtype, 300 + M, bias=(N % 256 == 0))
+    bq.set_path(bq.PATH_TCGEN05)
+    out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, dtype,
+                  bias=None if bb is None else dev_bf16(bb))
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bb)
+    assert_gemm_close(out, ref, f"tcgen05 dtype={dtype} {M}x{N}x{K}")
+
+
+def test_gemm_tcgen05_rejects_ineligible_shapes():
+    _, qa, sa, qw, sw, _ = make_problem(16, 320, 200, 128, 128, INT8, 1)
+    bq.set_path(bq.PATH_TCGEN05)
+    with pytest.raises(bq.BqError) as ei:       # K = 200: row stride not a multiple of 16
+        bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, INT8)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+    _, qa, sa, qw, sw, _ = make_problem(64, 256, 256, 64, 128, INT8, 2)
+    with pytest.raises(bq.BqError) as ei:       # block_n = 64
+        bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 64, 128, INT8)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+
+
 def test_gemm_strided_operands_and_output():
     M, N, K, bn, bk = 70, 200, 300, 128, 128
     _, qa, sa, qw, sw, _ = make_problem(M, N, K, bn, bk, INT8, 7)
@@ -240,8 +276,29 @@ def test_moe_layer_stages_vs_oracle():
     assert (np.abs(ov - comb_ref) <= bf16_ulp(np.maximum(np.abs(ov), np.abs(comb_ref)))).all()
 
 
-def test_grouped_gemm_leaves_rows_past_offsets_untouched():
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+def test_grouped_gemm_tcgen05_vs_oracle(dtype):
+    p = moe_problem(T=300, H=384, I=256, E=8, dtype=dtype, seed=33)
+    T, I, E, topk = p["T"], p["I"], p["E"], p["topk"]
+    off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), E)
+    o_ref, p_ref, _ = oracle.moe_permute(p["ids"], E)
+    qa, sa = bq.moe_quant_gather(dev_bf16(p["x"]), perm, topk, 128, dtype)
+    qx, sx = oracle.quant_act(p["x"], 128, dtype)
+    rows = p_ref // topk
+    bq.set_path(bq.PATH_TCGEN05)
+    y13 = bq.grouped_gemm(qa, sa, off, dev_u8(p["q13"]), dev_f32(p["s13"]), 128, 128,
+                          n_seam=I, dtype=dtype)
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    ref13 = oracle.grouped_gemm(qx[rows], sx[rows], o_ref, p["q13"], p["s13"], 128, 128, dtype,
+                                seam=I)
+    assert_gemm_close(y13, ref13, "tcgen05 grouped w13")
+
+
+@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05])
+def test_grouped_gemm_leaves_rows_past_offsets_untouched(path):
     p = moe_problem(T=50, H=128, I=128, E=4)
+    bq.set_path(path)
     off = np.array([0, 10, 10, 30, 60], np.int32)     # 60 of the 100 rows routed
     R = 100
     qa = np.random.default_rng(0).integers(-100, 100, (R, 128)).astype(np.int8).view(np.uint8)

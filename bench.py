@@ -1,0 +1,550 @@
+#!/usr/bin/env python
+"""Throughput of the block-scaled W8A8 linear layer (libbq) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bq|reference]
+                    [--workload decode|prefill|fp8|moe] [--no-sub]
+
+Prints ONE JSON line.  The headline workload is the decode linear layer:
+INT8, N = K = 4096, [128,128] weight blocks, token counts M in {1, 8, 32, 64};
+one step = for each M, the dynamic 1x128 activation quantisation followed by
+the block-scaled GEMM (bq_quant_act + bq_gemm, i.e. bq_linear).  Sixteen
+weight copies rotate (268 MB > the 126 MB L2), so every GEMM streams its
+weights from HBM.  `value` is whole-job algorithmic HBM bytes per second.
+Sub-workloads (prefill INT8 4096x14336x4096, FP8 e4m3 2048x4096x14336, and
+the INT8 MoE layer T=4096, E=8, top-2) report TOPS against the tensor roofline.
+
+Multi-GPU: the layer shards over tokens with no exchange (replicas), so each
+rank runs the same per-rank work ("scaling": "weak"); time is the max over
+ranks of CUDA-event time.  `--impl reference` times the CPU oracle (the
+plain C reference) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import bq_synth  # noqa: E402
+
+METRIC = "block-scaled W8A8 GEMM TOPS & weight GB/s; % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.n_gpus = n_gpus
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        elif torch.cuda.is_available():
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    mhz.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        loaded = [m for m in mhz if mx and m > 0.5 * mx] or mhz
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "samples": len(mhz), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------
+# helpers
+# --------------------------------------------------------------------------
+
+def cdiv(a, b):
+    return -(-a // b)
+
+
+def timed_graph_steps(graphs, steps, warmup, stream, dist):
+    """Replay graphs[i % len(graphs)] for warmup+steps; returns seconds of the
+    timed steps (CUDA events, max over ranks)."""
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        graphs[(warmup + i) % len(graphs)].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    return dist.max(e0.elapsed_time(e1) / 1e3)
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()                       # warm (allocations, attributes)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def quant_weights(w, dtype, bq):
+    q, s = bq.quant_weight(w, 128, 128, dtype)
+    return q, s
+
+
+# --------------------------------------------------------------------------
+# workloads (CUDA path)
+# --------------------------------------------------------------------------
+
+def bench_decode(args, dist, bq, peaks, stream):
+    N = K = 4096
+    Ms = bq_synth.DECODE_MS
+    NW = 16
+    dev = torch.device("cuda", torch.cuda.current_device())
+    Nb, Kb = cdiv(N, 128), cdiv(K, 128)
+    ws_q, ws_s = [], []
+    for i in range(NW):
+        w = bq_synth.weights(N, K, 0.02, 100 + i, device=dev)
+        q, s = quant_weights(w, bq.INT8, bq)
+        ws_q.append(q)
+        ws_s.append(s)
+        del w
+    xs = [bq_synth.activations(M, K, cfg.seed, cfg.n_outliers, cfg.outlier_scale, device=dev)
+          for M, cfg in zip(Ms, bq_synth.DECODE)]
+    outs = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms]
+    qa = [torch.empty(M, K, dtype=torch.uint8, device=dev) for M in Ms]
+    sa = [torch.empty(Kb, M, dtype=torch.float32, device=dev) for M in Ms]
+    gws = [bq.workspace(bq.gemm_workspace_size(M, N, K), dev) for M in Ms]
+    torch.cuda.synchronize()
+
+    def step(phase, quant=True, gemm=True):
+        def run():
+            for j, M in enumerate(Ms):
+                wi = (4 * phase + j) % NW
+                if quant:
+                    bq.quant_act(xs[j], 128, bq.INT8, q=qa[j], s=sa[j])
+                if gemm:
+                    bq.gemm(qa[j], sa[j], ws_q[wi], ws_s[wi], 128, 128, bq.INT8, out=outs[j],
+                            ws=gws[j])
+        return run
+
+    phases = NW // len(Ms)
+    graphs = [capture(step(p), stream) for p in range(phases)]
+    gemm_graphs = [capture(step(p, quant=False), stream) for p in range(phases)]
+    quant_graphs = [capture(step(p, gemm=False), stream) for p in range(phases)]
+
+    gemm_bytes = sum(N * K + 4 * Nb * Kb + M * K + 4 * M * Kb + 2 * M * N for M in Ms)
+    step_bytes = sum(N * K + 4 * Nb * Kb + 2 * M * K + 2 * M * N for M in Ms)
+    with Clocks(torch.cuda.current_device()) as clk:
+        t = timed_graph_steps(graphs, args.steps, args.warmup, stream, dist)
+        t_gemm = timed_graph_steps(gemm_graphs, args.steps, args.warmup, stream, dist)
+        t_quant = timed_graph_steps(quant_graphs, args.steps, args.warmup, stream, dist)
+    clocks = clk.summary()
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # activations from pinned memory, bq_linear, D2H of the outputs
+    hx = [x.cpu().pin_memory() for x in xs]
+    ho = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in Ms]
+    dx = [torch.empty_like(x, device=dev) for x in xs]
+    lws = bq.workspace(max(bq.linear_workspace_size(M, N, K) for M in Ms), dev)
+
+    def e2e(phase):
+        def run():
+            for j, M in enumerate(Ms):
+                wi = (4 * phase + j) % NW
+                dx[j].copy_(hx[j], non_blocking=True)
+                bq.linear(dx[j], ws_q[wi], ws_s[wi], 128, 128, bq.INT8, out=outs[j], ws=lws)
+                ho[j].copy_(outs[j], non_blocking=True)
+        return run
+
+    e2e_graphs = [capture(e2e(p), stream) for p in range(phases)]
+    t_e2e = timed_graph_steps(e2e_graphs, args.steps, args.warmup, stream, dist)
+
+    n = dist.world
+    value = n * args.steps * step_bytes / t / 1e9
+    gemm_launch_s = t_gemm / (args.steps * len(Ms))
+    achieved = gemm_bytes / len(Ms) / gemm_launch_s / 1e9
+    res = {
+        "value": value, "unit": "GB/s", "ms_per_step": 1e3 * t / args.steps,
+        "roofline": {"bound": "hbm", "kernel": "block-scaled GEMM (decode shapes)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes_per_launch": gemm_bytes / len(Ms),
+                     "avg_launch_us": 1e6 * gemm_launch_s},
+        "quant_us_per_launch": 1e6 * t_quant / (args.steps * len(Ms)),
+        "e2e": {"value": n * args.steps * step_bytes / t_e2e / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": sum(2 * M * K for M in Ms),
+                "d2h_bytes_per_step": sum(2 * M * N for M in Ms)},
+        "gpu_launches": args.steps * 2 * len(Ms),
+        "clocks": clocks,
+        "config": {"workload": "decode_int8_n4096_k4096_m1-8-32-64", "M": list(Ms), "N": N,
+                   "K": K, "block": [128, 128], "act_group": 128,
+                   "l2": "16 rotating weight copies (268 MB) > 126 MB L2",
+                   "parallelism": f"replicas x{n}"},
+        "dtype": "int8",
+        "gemm_path": "auto",
+    }
+    del graphs, gemm_graphs, quant_graphs, e2e_graphs
+    return res
+
+
+def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    M, N, K = cfg.M, cfg.N, cfg.K
+    wq, wsc = [], []
+    for i in range(n_rot):
+        w = bq_synth.weights(N, K, cfg.w_std, cfg.seed + 10 * i, device=dev)
+        q, s = quant_weights(w, cfg.dtype, bq)
+        wq.append(q)
+        wsc.append(s)
+        del w
+    xs = [bq_synth.activations(M, K, cfg.seed + i, cfg.n_outliers, cfg.outlier_scale,
+                               device=dev) for i in range(n_rot)]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    Kb = cdiv(K, 128)
+    qa = torch.empty(M, K, dtype=torch.uint8, device=dev)
+    sa = torch.empty(Kb, M, dtype=torch.float32, device=dev)
+    gws = bq.workspace(bq.gemm_workspace_size(M, N, K, 128, 128, cfg.dtype), dev)
+    torch.cuda.synchronize()
+
+    def step(i, quant=True):
+        def run():
+            if quant:
+                bq.quant_act(xs[i], 128, cfg.dtype, q=qa, s=sa)
+            bq.gemm(qa, sa, wq[i], wsc[i], 128, 128, cfg.dtype, out=out, ws=gws)
+        return run
+
+    graphs = [capture(step(i), stream) for i in range(n_rot)]
+    gemm_graphs = [capture(step(i, False), stream) for i in range(n_rot)]
+    with Clocks(torch.cuda.current_device()) as clk:
+        t = timed_graph_steps(graphs, args.steps, args.warmup, stream, dist)
+        t_gemm = timed_graph_steps(gemm_graphs, args.steps, args.warmup, stream, dist)
+    ops = 2.0 * M * N * K
+    peak = 2.0 * peaks["bf16_tflops"]
+    ach = ops / (t_gemm / args.steps) / 1e12
+    del graphs, gemm_graphs
+    return {"value": dist.world * args.steps * ops / t / 1e12, "unit": "TOPS",
+            "ms_per_step": 1e3 * t / args.steps,
+            "roofline": {"bound": "tensor", "kernel": "tcgen05 block-scaled GEMM",
+                         "achieved": ach, "peak": peak, "unit": "TFLOP/s" if cfg.dtype else
+                         "TOPS", "frac": ach / peak, "traffic": None,
+                         "peak_source": "2 x measured bf16 burst (8-bit dense = 2x bf16)",
+                         "avg_launch_us": 1e6 * t_gemm / args.steps},
+            "clocks": clk.summary(),
+            "config": {"workload": cfg.name, "M": M, "N": N, "K": K, "block": [128, 128],
+                       "l2": f"{n_rot} rotating weight/activation copies"},
+            "dtype": "fp8_e4m3" if cfg.dtype else "int8"}
+
+
+def bench_moe(args, dist, bq, peaks, stream):
+    cfg = bq_synth.MOE
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T, H, I, E, topk = cfg.T, cfg.H, cfg.I, cfg.E, cfg.topk
+    x = bq_synth.activations(T, H, cfg.seed, device=dev)
+    ids, tw = bq_synth.routing(T, E, topk, cfg.seed)
+    ids_d = torch.from_numpy(ids).to(dev)
+    tw_d = torch.from_numpy(tw).to(dev)
+    q13 = torch.empty(E, 2 * I, H, dtype=torch.uint8, device=dev)
+    s13 = torch.empty(E, 2 * cdiv(I, 128), cdiv(H, 128), dtype=torch.float32, device=dev)
+    q2 = torch.empty(E, H, I, dtype=torch.uint8, device=dev)
+    s2 = torch.empty(E, cdiv(H, 128), cdiv(I, 128), dtype=torch.float32, device=dev)
+    for e in range(E):
+        w13 = bq_synth.weights(2 * I, H, cfg.w_std, cfg.seed + 31 * e, device=dev)
+        for half in range(2):
+            q, s = bq.quant_weight(w13[half * I:(half + 1) * I].contiguous(), 128, 128, cfg.dtype)
+            q13[e, half * I:(half + 1) * I] = q
+            s13[e, half * cdiv(I, 128):(half + 1) * cdiv(I, 128)] = s
+        del w13
+        w2 = bq_synth.weights(H, I, cfg.w_std, cfg.seed + 31 * e + 1, device=dev)
+        q, s = bq.quant_weight(w2, 128, 128, cfg.dtype)
+        q2[e], s2[e] = q, s
+        del w2
+    R = T * topk
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(R, dtype=torch.int32, device=dev)
+    inv = torch.empty(R, dtype=torch.int32, device=dev)
+    qa = torch.empty(R, H, dtype=torch.uint8, device=dev)
+    sa = torch.empty(cdiv(H, 128), R, dtype=torch.float32, device=dev)
+    y13 = torch.empty(R, 2 * I, dtype=torch.bfloat16, device=dev)
+    qh = torch.empty(R, I, dtype=torch.uint8, device=dev)
+    sh = torch.empty(cdiv(I, 128), R, dtype=torch.float32, device=dev)
+    y2 = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    ws13 = bq.workspace(bq.grouped_gemm_workspace_size(R, 2 * I, H, E), dev)
+    torch.cuda.synchronize()
+    L = bq.lib()
+    st = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+
+    def layer(parts=("perm", "gather", "w13", "silu", "w2", "comb")):
+        def run():
+            if "perm" in parts:
+                bq._check(L.bq_moe_permute(ids_d.data_ptr(), T, topk, E, off.data_ptr(),
+                                           perm.data_ptr(), inv.data_ptr(), None, 0, st()))
+            if "gather" in parts:
+                bq.moe_quant_gather(x, perm, topk, 128, cfg.dtype, q=qa, s=sa)
+            if "w13" in parts:
+                bq.grouped_gemm(qa, sa, off, q13, s13, 128, 128, I, cfg.dtype, out=y13, ws=ws13)
+            if "silu" in parts:
+                bq.moe_silu_mul_quant(y13, I, 128, cfg.dtype, q=qh, s=sh)
+            if "w2" in parts:
+                bq.grouped_gemm(qh, sh, off, q2, s2, 128, 128, 0, cfg.dtype, out=y2, ws=ws13)
+            if "comb" in parts:
+                bq.moe_combine(y2, inv, tw_d, out=out)
+        return run
+
+    g = [capture(layer(), stream)]
+    gg = [capture(layer(("w13", "w2")), stream)]
+    steps = max(3, args.steps // 4)
+    with Clocks(torch.cuda.current_device()) as clk:
+        t = timed_graph_steps(g, steps, args.warmup, stream, dist)
+        t_g = timed_graph_steps(gg, steps, args.warmup, stream, dist)
+    ops = 2.0 * R * (2 * I) * H + 2.0 * R * H * I
+    peak = 2.0 * peaks["bf16_tflops"]
+    ach = ops / (t_g / steps) / 1e12
+    del g, gg
+    return {"value": dist.world * steps * ops / t / 1e12, "unit": "TOPS",
+            "ms_per_step": 1e3 * t / steps, "steps": steps,
+            "roofline": {"bound": "tensor", "kernel": "tcgen05 grouped GEMM (w13 + w2)",
+                         "achieved": ach, "peak": peak, "unit": "TOPS", "frac": ach / peak,
+                         "traffic": None, "avg_pair_us": 1e6 * t_g / steps},
+            "clocks": clk.summary(),
+            "config": {"workload": cfg.name, "T": T, "H": H, "I": I, "E": E, "topk": topk,
+                       "block": [128, 128], "routing": "softmax(N(0,1) logits) top-2"},
+            "dtype": "int8"}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_decode_sample(n_rows: int):
+    """One decode step restricted to the first n_rows weight rows: the oracle's
+    activation quantisation for M in {1,8,32,64} and its GEMM against an
+    [n_rows, 4096] weight slice.  Returns (seconds, algorithmic bytes)."""
+    import oracle
+    K = 4096
+    w = bq_synth.weights(n_rows, K, 0.02, 100).numpy()
+    qw, sw = oracle.quant_weight(w, 128, 128, oracle.INT8)
+    xs = [bq_synth.bf16_bits(bq_synth.activations(M, K, c.seed, c.n_outliers,
+                                                  c.outlier_scale))
+          for M, c in zip(bq_synth.DECODE_MS, bq_synth.DECODE)]
+    t0 = time.perf_counter()
+    for xb in xs:
+        qa, sa = oracle.quant_act(xb, 128, oracle.INT8)
+        oracle.gemm(qa, sa, qw, sw, 128, 128, oracle.INT8)
+    dt = time.perf_counter() - t0
+    Nb, Kb = cdiv(n_rows, 128), K // 128
+    nbytes = sum(n_rows * K + 4 * Nb * Kb + 2 * M * K + 2 * M * n_rows
+                 for M in bq_synth.DECODE_MS)
+    return dt, nbytes
+
+
+def cpu_baseline(seconds_target=20.0):
+    dt, nb = oracle_decode_sample(256)
+    rows = int(min(4096, max(128, 256 * seconds_target / max(dt, 1e-3) / 2)))
+    rows = max(128, rows // 128 * 128)
+    dt, nb = oracle_decode_sample(rows)
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one decode step (M in 1,8,32,64; K=4096) on the first {rows} of the "
+                      f"4096 weight rows; single-threaded C oracle; {dt:.1f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 256
+    for _ in range(args.warmup):
+        oracle_decode_sample(rows)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = oracle_decode_sample(rows)
+        tot_t += dt
+        tot_b += nb
+    v = tot_b / tot_t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "decode_int8_n4096_k4096_m1-8-32-64",
+                       "sample_rows": rows, "world_size": world},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: one decode step on {rows} of 4096 weight "
+                                       "rows, single-threaded C oracle"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="bq", choices=["bq", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fp8", "moe"])
+    ap.add_argument("--no-sub", action="store_true", help="skip the sub-workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import block_scaled_w8a8_b200 as bq
+    bq.lib()                         # fails loudly if the CUDA library is missing
+    dist = Dist(args.gpus)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        subs = {}
+        if args.workload == "decode":
+            head = bench_decode(args, dist, bq, peaks, stream)
+        elif args.workload == "prefill":
+            head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.PREFILL, 3)
+        elif args.workload == "fp8":
+            head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.FP8_LINEAR, 3)
+        else:
+            head = bench_moe(args, dist, bq, peaks, stream)
+        if not args.no_sub:
+            for name in ("prefill", "fp8", "moe"):
+                if name == args.workload:
+                    continue
+                torch.cuda.empty_cache()
+                if name == "prefill":
+                    subs[name] = bench_linear_big(args, dist, bq, peaks, stream,
+                                                  bq_synth.PREFILL, 3)
+                elif name == "fp8":
+                    subs[name] = bench_linear_big(args, dist, bq, peaks, stream,
+                                                  bq_synth.FP8_LINEAR, 3)
+                else:
+                    subs[name] = bench_moe(args, dist, bq, peaks, stream)
+    bq.check_device_status()
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
+        cpu = cpu_baseline()
+    if dist.rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": head["unit"],
+                "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
+                "data": "synthetic (seeded Gaussian activations with outlier channels; "
+                        "Gaussian weights block-quantised on the GPU)",
+                "config": head["config"], "roofline": head["roofline"],
+                "peaks_source": peak_src, "clocks": head["clocks"],
+                "e2e": head.get("e2e"), "gpu_launches": head.get("gpu_launches"),
+                "cpu_baseline": cpu, "workloads": subs}
+        for k in ("quant_us_per_launch", "gemm_path"):
+            if k in head:
+                line[k] = head[k]
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -210,10 +210,11 @@ bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_
   return ok();
 }
 
-bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, int64_t ldw,
-                  const float* sw, int64_t M, int64_t N, int64_t K, int64_t block_n,
-                  int64_t block_k, int dtype, const void* bias, void* out, int64_t ldo,
-                  void* workspace, size_t workspace_bytes, void* stream) {
+static bq_status gemm_impl(const void* qa, int64_t lda, const float* sa, const void* qw,
+                           int64_t ldw, const float* sw, int64_t M, int64_t N, int64_t K,
+                           int64_t block_n, int64_t block_k, int dtype, const void* bias,
+                           void* out, int64_t ldo, void* workspace, size_t workspace_bytes,
+                           void* stream, bool after_quant) {
   bq_status st = check_gemm_shape(M, N, K, block_n, block_k, dtype);
   if (st != BQ_OK) return st;
   BQ_CHECK_ARG(lda >= K && ldw >= K && ldo >= N, "leading dimensions too small");
@@ -236,12 +237,34 @@ bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, 
   a.offsets = nullptr; a.E = 1; a.w_expert_stride = 0; a.sw_expert_stride = 0;
   a.status = w;
   char why[256] = "";
-  const int rc = bq::run_gemm(a, g_path, workspace, workspace_bytes, as_stream(stream), why,
-                              sizeof(why));
+  const int rc = after_quant ? bq::run_gemm_after_quant(a, g_path, workspace, workspace_bytes,
+                                                        as_stream(stream), why, sizeof(why))
+                             : bq::run_gemm(a, g_path, workspace, workspace_bytes,
+                                            as_stream(stream), why, sizeof(why));
   if (rc == bq::kRunOk) return ok();
   if (rc == bq::kRunUnsupported) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
   if (rc == bq::kRunAlignment) return fail(BQ_ERR_ALIGNMENT, "%s", why);
   return fail(BQ_ERR_CUDA, "%s", why);
+}
+
+bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, int64_t ldw,
+                  const float* sw, int64_t M, int64_t N, int64_t K, int64_t block_n,
+                  int64_t block_k, int dtype, const void* bias, void* out, int64_t ldo,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_impl(qa, lda, sa, qw, ldw, sw, M, N, K, block_n, block_k, dtype, bias, out, ldo,
+                   workspace, workspace_bytes, stream, false);
+}
+
+// bq_linear workspace: [GEMM workspace (its counter region at offset 0)]
+// [activation codes M x ldq] [activation scales Kb x M].
+static void linear_layout(int64_t M, int64_t N, int64_t K, int64_t block_n, int64_t block_k,
+                          int dtype, size_t* gemm_bytes, size_t* q_off, size_t* s_off,
+                          size_t* total, int64_t* ldq) {
+  *ldq = (int64_t)round_up((size_t)K, 16);
+  *gemm_bytes = round_up(bq::gemm_workspace_bytes(M, N, K, block_n, block_k, dtype), 256);
+  *q_off = *gemm_bytes;
+  *s_off = *q_off + round_up((size_t)(M * *ldq), 256);
+  *total = *s_off + round_up((size_t)(cdiv(K, block_k) * M) * sizeof(float), 256);
 }
 
 bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_n,
@@ -249,11 +272,10 @@ bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t bloc
   bq_status st = check_gemm_shape(M, N, K, block_n, block_k, dtype);
   if (st != BQ_OK) return st;
   BQ_CHECK_ARG(bytes, "bytes must not be NULL");
-  const int64_t ldq = round_up((size_t)K, 16);
-  size_t b = round_up((size_t)(M * ldq), 256);
-  b += round_up((size_t)(cdiv(K, block_k) * M) * sizeof(float), 256);
-  b += bq::gemm_workspace_bytes(M, N, K, block_n, block_k, dtype);
-  *bytes = b;
+  size_t g, qo, so, tot;
+  int64_t ldq;
+  linear_layout(M, N, K, block_n, block_k, dtype, &g, &qo, &so, &tot, &ldq);
+  *bytes = tot;
   return ok();
 }
 
@@ -267,27 +289,22 @@ bq_status bq_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void
   if (M == 0 || N == 0) return ok();
   BQ_CHECK_ARG(out, "out must not be NULL");
   BQ_CHECK_ARG(K == 0 || (x && qw && sw), "x, qw and sw must not be NULL");
-  size_t need = 0;
-  st = bq_linear_workspace_size(M, N, K, block_n, block_k, dtype, &need);
-  if (st != BQ_OK) return st;
+  size_t g, qo, so, need;
+  int64_t ldq;
+  linear_layout(M, N, K, block_n, block_k, dtype, &g, &qo, &so, &need, &ldq);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(BQ_ERR_WORKSPACE, "bq_linear needs %zu workspace bytes, got %zu", need,
                 workspace ? workspace_bytes : (size_t)0);
-  const int64_t ldq = round_up((size_t)K, 16);
   uint8_t* base = static_cast<uint8_t*>(workspace);
-  void* q = base;
-  size_t off = round_up((size_t)(M * ldq), 256);
-  float* s = reinterpret_cast<float*>(base + off);
-  off += round_up((size_t)(cdiv(K, block_k) * M) * sizeof(float), 256);
-  void* gws = base + off;
-  const size_t gws_bytes = workspace_bytes - off;
+  void* q = base + qo;
+  float* s = reinterpret_cast<float*>(base + so);
   if (K > 0) {
     BQ_CHECK_CUDA(bq::launch_quant_act(x, M, K, ldx, nullptr, 1, block_k, dtype, q, ldq, s,
                                        as_stream(stream)),
                   "quant_act launch");
   }
-  return bq_gemm(q, ldq, s, qw, ldw, sw, M, N, K, block_n, block_k, dtype, bias, out, ldo,
-                 gws, gws_bytes, stream);
+  return gemm_impl(q, ldq, s, qw, ldw, sw, M, N, K, block_n, block_k, dtype, bias, out, ldo,
+                   base, g, stream, true);
 }
 
 bq_status bq_moe_permute_workspace_size(int64_t T, int64_t topk, int64_t E, size_t* bytes) {

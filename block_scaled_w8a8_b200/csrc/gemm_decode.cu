@@ -1,0 +1,448 @@
+// gemm_decode.cu -- block-scaled GEMM for few tokens (decode), weight-streaming.
+//
+// Same contraction as the other GEMMs (block-wise INT8 page, sections 2 and 4;
+// blockwise FP8 of the SGLang quantization doc), for M <= 128 tokens and
+// block_n = block_k = 128.  With so few tokens the layer is bound by reading
+// the weights once from HBM, so the kernel is organised around that stream:
+//
+//  * swap-AB: the 128 weight rows of a tile are the MMA's M dimension and the
+//    tokens (padded to NT = 16/32/64/128) its N dimension, so no MMA rows are
+//    wasted on padding tokens;  D[n, t] = sum_k W[n, k] * A[t, k];
+//  * split-K: CTA (tile, split) streams the K-blocks [kb0, kb1) of one 128-row
+//    weight tile through a TMA ring (16 KB per K-block, all loads in flight at
+//    once); the grid has ~2 CTAs per SM so every SM keeps loads in flight;
+//  * per-K-block promotion in the epilogue warps (one weight row per thread,
+//    one token per TMEM column): acc[t] += P * sa[kb][t] * sw[tile][kb];
+//  * split partials go to a workspace; the last CTA to finish a tile sums
+//    them in split order (deterministic), adds the bias, writes bf16 and
+//    resets the tile's arrival counter.  The counters live in the first
+//    kDecodeCounterBytes of the workspace (a fixed place, whatever the shape),
+//    so a workspace whose counter region starts zeroed stays usable by any
+//    sequence of calls; the partials after it need no initialisation;
+//  * programmatic dependent launch: the weight loads are issued before
+//    griddepcontrol.wait, so they overlap the activation quantiser that
+//    produces this kernel's A operand.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstdio>
+
+#include "bq_common.cuh"
+#include "bq_internal.h"
+#include "gemm_decode.h"
+#include "sm100.cuh"
+
+namespace bq {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BN_W = 128;   // weight rows per tile (MMA M)
+constexpr int BK = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kMaxSplitKb = 32;  // K-blocks per split (their act scales sit in smem)
+
+struct DecParams {
+  const float* sa;       // [Kb][M]
+  const float* sw;       // [Nb][Kb]
+  int64_t M, N, K, Kb;
+  int splits;
+  const uint16_t* bias;
+  uint16_t* out; int64_t ldo;
+  float* part;           // [splits][M][N] (splits > 1)
+  unsigned* counters;    // [n_tiles]
+  unsigned* status;
+};
+
+template <int NT>
+struct DSmem {
+  static constexpr uint32_t kW = BN_W * BK, kA = NT * BK;
+  static constexpr uint32_t kStage = kW + kA;
+  static constexpr uint32_t kStages_ = kStages * kStage;
+  static constexpr uint32_t kSa = kMaxSplitKb * NT * 4;
+  static constexpr uint32_t kTotal = 1024 + kStages_ + kSa + (2 * kStages + 5) * 8 + 16;
+};
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <int DT>
+__device__ __forceinline__ float pval(uint32_t b) {
+  if constexpr (DT == kInt8) return __int2float_rn((int)b);
+  else return __uint_as_float(b);
+}
+
+// 32 lanes x 16 columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+template <int NT>
+constexpr uint32_t tmem_cols() {
+  return (2 * NT) <= 32 ? 32 : (2 * NT) <= 64 ? 64 : (2 * NT) <= 128 ? 128 : 256;
+}
+
+template <int DT, int NT>
+__global__ void __launch_bounds__(kThreads)
+gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
+                   const DecParams p) {
+  using L = DSmem<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* sa_s = reinterpret_cast<float*>(smem + L::kStages_);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStages_ + L::kSa);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = bars + 2 * kStages + 2;
+  uint64_t* drain = bars + 2 * kStages + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int kb0 = (int)((int64_t)split * p.Kb / p.splits);
+  const int kb1 = (int)((int64_t)(split + 1) * p.Kb / p.splits);
+  const int nkb = kb1 - kb0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull[b]), 1);
+      mbar_init(smem_u32(&tempty[b]), 4);
+    }
+    mbar_init(smem_u32(&drain[0]), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), tmem_cols<NT>());
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmW);
+      tma_prefetch_desc(&tmA);
+    }
+    // weights first (independent of the preceding kernel), then activations
+    const int first = min(nkb, kStages);
+    if (lane == 0) {
+      for (int i = 0; i < first; ++i) {
+        mbar_arrive_expect_tx(smem_u32(&full[i]), L::kStage);
+        tma_load_2d(smem_u32(smem + i * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
+                    smem_u32(&full[i]));
+      }
+    }
+    grid_dep_wait();
+    if (lane == 0) {
+      for (int i = 0; i < first; ++i)
+        tma_load_2d(smem_u32(smem + i * L::kStage + L::kW), &tmA, (kb0 + i) * BK, 0,
+                    smem_u32(&full[i]));
+    }
+    bool ok = true;
+    int issued_parity[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) issued_parity[s] = s < first ? 0 : -1;
+    for (int i = first; i < nkb && ok; ++i) {
+      const int stage = i % kStages;
+      const uint32_t phase = (uint32_t)((i / kStages) & 1);
+      if (!warp_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.status, 0x401u)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kStage);
+        tma_load_2d(smem_u32(smem + stage * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
+                    smem_u32(&full[stage]));
+        tma_load_2d(smem_u32(smem + stage * L::kStage + L::kW), &tmA, (kb0 + i) * BK, 0,
+                    smem_u32(&full[stage]));
+      }
+      issued_parity[stage] = (int)phase;
+    }
+    if (!ok) {
+      for (int s = 0; s < kStages; ++s) {
+        if (issued_parity[s] < 0) continue;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(&full[s]), (uint32_t)issued_parity[s]) &&
+               globaltimer() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t idesc = instr_desc<DT>(BN_W, NT);
+    bool issued_any = false, ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const int stage = i % kStages;
+      const uint32_t phase = (uint32_t)((i / kStages) & 1);
+      const uint32_t buf = i & 1, tround = (uint32_t)(i >> 1);
+      if (!warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag, p.status, 0x402u) ||
+          !warp_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x403u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t d = tmem_base + buf * NT;
+        const uint64_t a0 = smem_desc_k128(smem_u32(smem + stage * L::kStage));
+        const uint64_t b0 = smem_desc_k128(smem_u32(smem + stage * L::kStage + L::kW));
+#pragma unroll
+        for (int j = 0; j < BK / 32; ++j)
+          mma<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+        mma_commit(smem_u32(&empty[stage]));
+        mma_commit(smem_u32(&tfull[buf]));
+      }
+      __syncwarp();
+      issued_any = true;
+    }
+    if (!ok && issued_any) {
+      // wait (bounded) for the MMAs already issued before TMEM is freed
+      if (lane == 0) mma_commit(smem_u32(&drain[0]));
+      __syncwarp();
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(smem_u32(&drain[0]), 0) && globaltimer() - t0 < 100000000ull) {
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;                       // TMEM lane quadrant of this warp
+    const int et = threadIdx.x - 64;              // 0..127
+    const int64_t n = (int64_t)tile * BN_W + 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    grid_dep_wait();                              // sa is written by the quantiser
+    for (int idx = et; idx < nkb * NT; idx += 128) {
+      const int kbl = idx / NT, t = idx % NT;
+      sa_s[idx] = (t < p.M) ? p.sa[(int64_t)(kb0 + kbl) * p.M + t] : 0.f;
+    }
+    named_bar(1, 128);
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const uint32_t buf = i & 1, tround = (uint32_t)(i >> 1);
+      const float swv = __ldg(p.sw + (int64_t)tile * p.Kb + kb0 + i);
+      if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x404u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < NT / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem_base + lane_base + buf * NT + 16 * c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * c + j;
+          acc[t] = fmaf(pval<DT>(r[j]), sa_s[i * NT + t] * swv, acc[t]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+    }
+    (void)ok;
+    named_bar(1, 128);                 // all four epilogue warps decide together
+    if (!*abort_flag) {
+      const bool n_ok = n < p.N;
+      if (p.splits == 1) {
+        if (n_ok) {
+          const float b = p.bias ? bf16_bits_to_float(p.bias[n]) : 0.f;
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            if (t < p.M) p.out[(int64_t)t * p.ldo + n] = float_to_bf16_bits(acc[t] + b);
+        }
+      } else {
+        if (n_ok) {
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            if (t < p.M) p.part[((int64_t)split * p.M + t) * p.N + n] = acc[t];
+        }
+        __threadfence();
+        named_bar(1, 128);
+        if (et == 0) {
+          const unsigned old = atomicAdd(&p.counters[tile], 1u);
+          *last_flag = (old == (unsigned)(p.splits - 1)) ? 1 : 0;
+        }
+        named_bar(1, 128);
+        if (*last_flag) {
+          __threadfence();
+          if (n_ok) {
+            const float b = p.bias ? bf16_bits_to_float(p.bias[n]) : 0.f;
+            for (int t = 0; t < (int)p.M; ++t) {
+              float sum = 0.f;
+              for (int s = 0; s < p.splits; ++s)
+                sum += __ldcg(p.part + ((int64_t)s * p.M + t) * p.N + n);
+              p.out[(int64_t)t * p.ldo + n] = float_to_bf16_bits(sum + b);
+            }
+          }
+          if (et == 0) p.counters[tile] = 0u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols<NT>());
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn enc() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+bool tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t ld,
+          uint32_t box_rows) {
+  if (!enc()) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {ld};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  return enc()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, v = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+  return v > 0 ? v : 148;
+}
+
+template <int DT, int NT>
+cudaError_t launch_nt(const GemmArgs& a, const DecodePlan& plan, void* ws, bool pdl,
+                      cudaStream_t st) {
+  using L = DSmem<NT>;
+  auto kern = gemm_decode_kernel<DT, NT>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tW, tA;
+  if (!tmap(&tW, a.qw, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.ldw, BN_W) ||
+      !tmap(&tA, a.qa, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.lda, NT))
+    return cudaErrorInvalidValue;
+  DecParams p;
+  p.sa = a.sa; p.sw = a.sw;
+  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK;
+  p.splits = plan.splits;
+  p.bias = static_cast<const uint16_t*>(a.bias);
+  p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.counters = plan.splits > 1 ? reinterpret_cast<unsigned*>(w) : nullptr;
+  p.part = plan.splits > 1 ? reinterpret_cast<float*>(w + kDecodeCounterBytes) : nullptr;
+  p.status = a.status;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)plan.tiles, (unsigned)plan.splits, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kTotal;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tW, tA, p);
+}
+
+template <int DT>
+cudaError_t launch_dt(const GemmArgs& a, const DecodePlan& plan, void* ws, bool pdl,
+                      cudaStream_t st) {
+  switch (plan.nt) {
+    case 16: return launch_nt<DT, 16>(a, plan, ws, pdl, st);
+    case 32: return launch_nt<DT, 32>(a, plan, ws, pdl, st);
+    case 64: return launch_nt<DT, 64>(a, plan, ws, pdl, st);
+    default: return launch_nt<DT, 128>(a, plan, ws, pdl, st);
+  }
+}
+
+}  // namespace
+
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
+  DecodePlan d;
+  d.nt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  d.tiles = (N + BN_W - 1) / BN_W;
+  const int64_t Kb = (K + BK - 1) / BK;
+  // about two CTAs per SM, at most kMaxSplitKb K-blocks per split
+  int64_t s = std::max<int64_t>(1, (2 * 148 + d.tiles - 1) / d.tiles);
+  s = std::min<int64_t>(s, Kb);
+  s = std::max<int64_t>(s, (Kb + kMaxSplitKb - 1) / kMaxSplitKb);
+  s = std::min<int64_t>(s, 65535);
+  d.splits = (int)s;
+  d.part_bytes = d.splits > 1 ? (size_t)d.splits * (size_t)M * (size_t)N * 4u : 0u;
+  d.part_bytes = (d.part_bytes + 255) / 256 * 256;
+  d.ws_bytes = d.splits > 1 ? kDecodeCounterBytes + d.part_bytes : 0u;
+  return d;
+}
+
+bool decode_supported(const GemmArgs& a, char* why, size_t n) {
+  auto no = [&](const char* msg) {
+    if (why) snprintf(why, n, "decode path: %s", msg);
+    return false;
+  };
+  if (a.offsets) return no("dense problems only");
+  if (a.M > 128) return no("at most 128 tokens");
+  if (a.bn != 128 || a.bk != 128) return no("needs block_n = block_k = 128");
+  if (a.K < 1) return no("needs K >= 1");
+  if (a.lda % 16 != 0 || a.ldw % 16 != 0) return no("row strides must be multiples of 16 bytes");
+  if ((reinterpret_cast<uintptr_t>(a.qa) & 15) || (reinterpret_cast<uintptr_t>(a.qw) & 15))
+    return no("operands must be 16-byte aligned");
+  if (a.N > INT32_MAX || a.K > INT32_MAX) return no("sizes exceed int32");
+  const int64_t tiles = (a.N + BN_W - 1) / BN_W;
+  if (tiles * 4 > (int64_t)kDecodeCounterBytes) return no("N too large for the counter region");
+  if (!enc()) return no("cuTensorMapEncodeTiled is unavailable");
+  return true;
+}
+
+cudaError_t launch_gemm_decode(const GemmArgs& a, void* ws, bool pdl, cudaStream_t st) {
+  if (a.M == 0 || a.N == 0) return cudaSuccess;
+  const DecodePlan plan = decode_plan(a.M, a.N, a.K);
+  (void)num_sms;
+  if (a.dtype == kInt8) return launch_dt<kInt8>(a, plan, ws, pdl, st);
+  return launch_dt<kFp8>(a, plan, ws, pdl, st);
+}
+
+}  // namespace bq

@@ -1,0 +1,30 @@
+// gemm_decode.h -- the few-token (decode) weight-streaming GEMM.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "bq_internal.h"
+
+namespace bq {
+
+// Arrival counters occupy the first 64 KiB of a decode workspace (one per
+// 128-row weight tile, so N <= 2^21 rows); the split partials follow.
+constexpr size_t kDecodeCounterBytes = 65536;
+
+struct DecodePlan {
+  int nt;              // token tile (MMA N): 16, 32, 64 or 128
+  int64_t tiles;       // 128-row weight tiles
+  int splits;          // K splits per tile
+  size_t part_bytes;   // fp32 split partials
+  size_t ws_bytes;     // counter region + partials (0 if splits == 1)
+};
+
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K);
+bool decode_supported(const GemmArgs& a, char* why, size_t n);
+// pdl: launch as a programmatic dependent of the preceding kernel (which must
+// not write the weights).  ws: zero-filled workspace of plan.ws_bytes.
+cudaError_t launch_gemm_decode(const GemmArgs& a, void* ws, bool pdl, cudaStream_t st);
+
+}  // namespace bq

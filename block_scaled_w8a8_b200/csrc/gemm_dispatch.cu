@@ -2,17 +2,24 @@
 //
 //   SIMT     generic CUDA-core kernel: any shape, stride, block size.
 //   TCGEN05  TMA + tcgen05 kernel: block_n = block_k = 128, 16-byte strides.
-// AUTO takes the tensor-core kernel whenever it applies and M is large
-// enough to fill an MMA tile, else the CUDA-core kernel.
+//   DECODE   swap-AB split-K weight-streaming tcgen05 kernel, M <= 128.
+// AUTO: M <= 128 -> DECODE, larger M -> TCGEN05, when they apply; otherwise
+// the CUDA-core kernel.
 #include <cstdio>
 
 #include "../../include/bq.h"
 #include "gemm_paths.h"
+#include "gemm_decode.h"
 #include "gemm_tc.h"
 
 namespace bq {
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int) { return 0; }
+constexpr int64_t kDecodeMaxRows = 128;
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t bn, int64_t bk, int) {
+  if (M < 1 || M > kDecodeMaxRows || N < 1 || K < 1 || bn != 128 || bk != 128) return 0;
+  return decode_plan(M, N, K).ws_bytes;
+}
 
 size_t grouped_workspace_bytes(int64_t, int64_t, int64_t, int64_t, int64_t, int64_t, int) {
   return 0;
@@ -36,16 +43,32 @@ static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
   return kRunOk;
 }
 
-constexpr int64_t kTcMinRows = 65;
+static int run_decode(const GemmArgs& a, void* ws, size_t ws_bytes, bool pdl, cudaStream_t st,
+                      char* why, size_t n) {
+  const size_t need = decode_plan(a.M, a.N, a.K).ws_bytes;
+  if (need > 0 && (ws == nullptr || ws_bytes < need)) {
+    snprintf(why, n, "decode path needs %zu workspace bytes, got %zu", need, ws_bytes);
+    return kRunUnsupported;
+  }
+  cudaError_t e = launch_gemm_decode(a, ws, pdl, st);
+  if (e != cudaSuccess) {
+    snprintf(why, n, "decode GEMM launch: %s", cudaGetErrorString(e));
+    return kRunCuda;
+  }
+  return kRunOk;
+}
 
-int run_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cudaStream_t st, char* why,
-             size_t why_len) {
-  (void)ws;
-  (void)ws_bytes;
+static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes, bool pdl,
+                          cudaStream_t st, char* why, size_t why_len) {
   switch (path) {
     case BQ_PATH_AUTO:
-      if (a.M >= kTcMinRows && tc_supported(a, nullptr, 0)) return run_tc(a, st, why, why_len);
+      if (a.M <= kDecodeMaxRows && decode_supported(a, nullptr, 0))
+        return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
+      if (a.M > kDecodeMaxRows && tc_supported(a, nullptr, 0)) return run_tc(a, st, why, why_len);
       return run_simt(a, st, why, why_len);
+    case BQ_PATH_DECODE:
+      if (!decode_supported(a, why, why_len)) return kRunUnsupported;
+      return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
     case BQ_PATH_SIMT:
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
@@ -55,6 +78,16 @@ int run_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cudaStream_
       snprintf(why, why_len, "kernel path %d is not available in this build", path);
       return kRunUnsupported;
   }
+}
+
+int run_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cudaStream_t st, char* why,
+             size_t why_len) {
+  return dispatch_dense(a, path, ws, ws_bytes, false, st, why, why_len);
+}
+
+int run_gemm_after_quant(const GemmArgs& a, int path, void* ws, size_t ws_bytes,
+                         cudaStream_t st, char* why, size_t why_len) {
+  return dispatch_dense(a, path, ws, ws_bytes, true, st, why, why_len);
 }
 
 int run_grouped_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cudaStream_t st,

@@ -19,6 +19,10 @@ size_t grouped_workspace_bytes(int64_t R, int64_t N, int64_t K, int64_t E, int64
 // failure writes a reason into `why`.
 int run_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cudaStream_t st,
              char* why, size_t why_len);
+// The GEMM half of bq_linear: like run_gemm, but a decode-path launch may
+// start as a programmatic dependent of the activation quantiser before it.
+int run_gemm_after_quant(const GemmArgs& a, int path, void* ws, size_t ws_bytes,
+                         cudaStream_t st, char* why, size_t why_len);
 int run_grouped_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cudaStream_t st,
                      char* why, size_t why_len);
 

@@ -92,6 +92,9 @@ quant_rows_kernel(const uint16_t* __restrict__ x, int64_t M_out, int64_t K, int6
                   const int32_t* __restrict__ perm, int64_t topk, int64_t gk, int64_t I_half,
                   uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
                   uint16_t* __restrict__ h_out, bool vec_in, bool vec_out) {
+  // let a programmatically dependent GEMM start streaming its weights now; it
+  // waits (griddepcontrol.wait) before reading what this kernel writes
+  asm volatile("griddepcontrol.launch_dependents;");
   const int lane = threadIdx.x & 31;
   const int64_t Kb = (K + gk - 1) / gk;
   const int64_t n_groups = M_out * Kb;

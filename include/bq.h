@@ -175,9 +175,12 @@ bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_
  * bias: bf16 [N] or NULL; out: bf16 [M, N] (row stride ldo >= N).
  * block_k <= 65536 keeps INT8 block partials exact in int32.
  * workspace: device memory of at least bq_gemm_workspace_size bytes (may be
- *   NULL when that size is 0).  Its first use must see it zero-filled; every
- *   successful call leaves it zero-filled again.  Calls sharing one
- *   workspace must not overlap on the GPU.
+ *   NULL when that size is 0).  Its first 64 KiB hold arrival counters: they
+ *   must be zero before the workspace is first used, and every completed
+ *   call leaves them zero again, whatever the shape, so one workspace can
+ *   serve any sequence of calls.  The rest needs no initialisation.  Calls
+ *   sharing one workspace must not overlap on the GPU; after a call that
+ *   reported a device error, zero the counter region again.
  * Block-wise INT8 page sections 2 and 4 (apply_w8a8_block_int8_linear with
  * input_scale=None, after the activation quantisation); blockwise FP8 of the
  * SGLang quantization doc. */
@@ -186,7 +189,8 @@ bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, 
                   int64_t block_k, int dtype, const void* bias, void* out, int64_t ldo,
                   void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace for bq_linear: the activation codes and scales plus bq_gemm's. */
+/* Workspace for bq_linear: bq_gemm's workspace (at offset 0, so the counter
+ * rule above applies) followed by the activation codes and scales. */
 bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_n,
                                    int64_t block_k, int dtype, size_t* bytes);
 

@@ -158,6 +158,76 @@ def test_gemm_tcgen05_rejects_ineligible_shapes():
     assert ei.value.status == bq.ERR_UNSUPPORTED
 
 
+DECODE_SHAPES = [
+    # M, N, K
+    (1, 640, 1008),      # 5 weight tiles x 8 splits of one K-block each
+    (8, 4096, 4096),     # the decode workload at M = 8
+    (16, 256, 512),
+    (17, 384, 2048),     # token count not a multiple of 16
+    (32, 1000, 1024),    # ragged last weight tile
+    (64, 640, 4096),
+    (100, 256, 1008),
+    (128, 512, 640),
+]
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+def test_gemm_decode_vs_oracle(dtype, M, N, K):
+    _, qa, sa, qw, sw, bb = make_problem(M, N, K, 128, 128, dtype, 500 + M, bias=(M % 2 == 1))
+    bq.set_path(bq.PATH_DECODE)
+    args = (dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, dtype)
+    bias = None if bb is None else dev_bf16(bb)
+    out1 = bq.gemm(*args, bias=bias)
+    out2 = bq.gemm(*args, bias=bias)     # the workspace must have reset itself
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bb)
+    assert_gemm_close(out1, ref, f"decode dtype={dtype} {M}x{N}x{K}")
+    assert torch.equal(out1, out2), "split-K reduction is not deterministic"
+
+
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_linear_decode_path_with_dependent_launch(M):
+    N = K = 4096
+    xb = act_bits(M, K, 40 + M, 41, 30.0)
+    w = bq_synth.weights(N, K, 0.02, 40 + M).numpy()
+    qw, sw = oracle.quant_weight(w, 128, 128, INT8)
+    x = dev_bf16(xb)
+    qw_d, sw_d = dev_u8(qw), dev_f32(sw)
+    outs = [bq.linear(x, qw_d, sw_d, 128, 128, INT8) for _ in range(3)]
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    qa, sa = oracle.quant_act(xb, 128, INT8)
+    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, INT8)
+    assert_gemm_close(outs[0], ref, f"linear decode M={M}")
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
+def test_linear_decode_in_cuda_graph():
+    M, N, K = 32, 1024, 2048
+    xb = act_bits(M, K, 77, 20, 30.0)
+    w = bq_synth.weights(N, K, 0.02, 77).numpy()
+    qw, sw = oracle.quant_weight(w, 128, 128, INT8)
+    x, qw_d, sw_d = dev_bf16(xb), dev_u8(qw), dev_f32(sw)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = bq.workspace(bq.linear_workspace_size(M, N, K), "cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        bq.linear(x, qw_d, sw_d, out=out, ws=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        bq.linear(x, qw_d, sw_d, out=out, ws=ws)
+    out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    qa, sa = oracle.quant_act(xb, 128, INT8)
+    assert_gemm_close(out, oracle.gemm(qa, sa, qw, sw, 128, 128, INT8), "graph replay")
+
+
 def test_gemm_strided_operands_and_output():
     M, N, K, bn, bk = 70, 200, 300, 128, 128
     _, qa, sa, qw, sw, _ = make_problem(M, N, K, bn, bk, INT8, 7)

@@ -49,6 +49,8 @@ DECLS = {
     "bq_gemm_workspace_size": (_INT, [_I64, _I64, _I64, _I64, _I64, _INT, _SZP]),
     "bq_gemm": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _I64, _I64, _INT, _P, _P,
                        _I64, _P, _SZ, _P]),
+    "bq_gemm_decode_noalloc": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _I64, _I64,
+                                      _INT, _P, _P, _I64, _P]),
     "bq_linear_workspace_size": (_INT, [_I64, _I64, _I64, _I64, _I64, _INT, _SZP]),
     "bq_linear": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I64, _I64, _INT, _P, _P,
                          _I64, _P, _SZ, _P]),
@@ -222,6 +224,22 @@ def gemm(qa, sa, qw, sw, block_n=128, block_k=128, dtype=INT8, bias=None, out=No
                          _cuda(sw, "sw"), M, N, K, block_n, block_k, dtype,
                          _opt(bias, "bias"), _cuda(out, "out"), _ld(out), _opt(ws, "ws"),
                          0 if ws is None else ws.numel(), _P(_stream(qa.device))))
+    return out
+
+
+def gemm_decode_noalloc(qa, sa, qw, sw, block_n=128, block_k=128, dtype=INT8, bias=None,
+                        out=None):
+    """bq_gemm on the decode kernel with the library's fixed scratch: no
+    workspace, no device allocation inside the call (for callers that cannot
+    allocate).  Overlapping calls race on the shared scratch."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qa.device)
+    _check(lib().bq_gemm_decode_noalloc(_cuda(qa, "qa"), _ld(qa), _cuda(sa, "sa"),
+                                        _cuda(qw, "qw"), _ld(qw), _cuda(sw, "sw"), M, N, K,
+                                        block_n, block_k, dtype, _opt(bias, "bias"),
+                                        _cuda(out, "out"), _ld(out), _P(_stream(qa.device))))
     return out
 
 

@@ -11,6 +11,7 @@
 #include "../../include/bq.h"
 #include "bq_common.cuh"
 #include "bq_internal.h"
+#include "gemm_decode.h"
 #include "gemm_paths.h"
 
 namespace {
@@ -265,6 +266,47 @@ static void linear_layout(int64_t M, int64_t N, int64_t K, int64_t block_n, int6
   *q_off = *gemm_bytes;
   *s_off = *q_off + round_up((size_t)(M * *ldq), 256);
   *total = *s_off + round_up((size_t)(cdiv(K, block_k) * M) * sizeof(float), 256);
+}
+
+bq_status bq_gemm_decode_noalloc(const void* qa, int64_t lda, const float* sa, const void* qw,
+                                 int64_t ldw, const float* sw, int64_t M, int64_t N, int64_t K,
+                                 int64_t block_n, int64_t block_k, int dtype, const void* bias,
+                                 void* out, int64_t ldo, void* stream) {
+  bq_status st = check_gemm_shape(M, N, K, block_n, block_k, dtype);
+  if (st != BQ_OK) return st;
+  BQ_CHECK_ARG(lda >= K && ldw >= K && ldo >= N, "leading dimensions too small");
+  if (M == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(out && qa && sa && qw && sw, "qa, sa, qw, sw and out must not be NULL");
+  unsigned* w = nullptr;
+  st = status_word(&w);
+  if (st != BQ_OK) return st;
+  bq::GemmArgs a{};
+  a.qa = qa; a.lda = lda; a.sa = sa; a.sa_rows = M;
+  a.qw = qw; a.ldw = ldw; a.sw = sw;
+  a.M = M; a.N = N; a.K = K; a.bn = block_n; a.bk = block_k; a.seam = 0;
+  a.Nbs = cdiv(N, block_n);
+  a.dtype = dtype; a.bias = bias; a.out = out; a.ldo = ldo;
+  a.offsets = nullptr; a.E = 1; a.w_expert_stride = 0; a.sw_expert_stride = 0;
+  a.status = w;
+  char why[256] = "";
+  if (!bq::decode_supported(a, why, sizeof(why))) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
+  const bq::DecodePlan plan = bq::decode_plan(M, N, K);
+  if (plan.ws_bytes > bq::kNoAllocScratchBytes)
+    return fail(BQ_ERR_UNSUPPORTED,
+                "this problem needs %zu bytes of scratch; the fixed scratch of "
+                "bq_gemm_decode_noalloc holds %zu (use bq_gemm with a workspace)",
+                plan.ws_bytes, bq::kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  BQ_CHECK_CUDA(bq::noalloc_scratch(&scratch), "static scratch address");
+  if (plan.splits > 1) {
+    // arrival counters must start at zero; the partials need no clearing
+    BQ_CHECK_CUDA(cudaMemsetAsync(scratch, 0, (size_t)plan.tiles * sizeof(unsigned),
+                                  as_stream(stream)),
+                  "scratch counter clear");
+  }
+  BQ_CHECK_CUDA(bq::launch_gemm_decode(a, scratch, false, as_stream(stream)),
+                "decode GEMM launch");
+  return ok();
 }
 
 bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_n,

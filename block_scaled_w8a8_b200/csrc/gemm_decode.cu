@@ -26,6 +26,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <mutex>
 
 #include "bq_common.cuh"
 #include "bq_internal.h"
@@ -435,6 +436,33 @@ bool decode_supported(const GemmArgs& a, char* why, size_t n) {
   if (tiles * 4 > (int64_t)kDecodeCounterBytes) return no("N too large for the counter region");
   if (!enc()) return no("cuTensorMapEncodeTiled is unavailable");
   return true;
+}
+
+// Scratch for bq_gemm_decode_noalloc: the decode kernel's arrival counters
+// (first kDecodeCounterBytes) and split partials, in a fixed device array so
+// that callers which cannot allocate device memory can still run the split-K
+// decode GEMM.  Every GPU that loads libbq holds these 16 MiB until the
+// process exits.  All calls share it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t noalloc_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[kMaxScratchDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    // The symbol's name is only a host-side handle: ask the runtime for the
+    // array's address on the current device, once per device.
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }
 
 cudaError_t launch_gemm_decode(const GemmArgs& a, void* ws, bool pdl, cudaStream_t st) {

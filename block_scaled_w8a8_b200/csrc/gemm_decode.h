@@ -23,6 +23,13 @@ struct DecodePlan {
 
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K);
 bool decode_supported(const GemmArgs& a, char* why, size_t n);
+// Fixed scratch of bq_gemm_decode_noalloc (counter region included).
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+constexpr int kMaxScratchDevices = 64;
+// Device address of that scratch on the current device (looked up on the
+// first call per device with cudaGetSymbolAddress).
+cudaError_t noalloc_scratch(void** ptr);
+
 // pdl: launch as a programmatic dependent of the preceding kernel (which must
 // not write the weights).  ws: zero-filled workspace of plan.ws_bytes.
 cudaError_t launch_gemm_decode(const GemmArgs& a, void* ws, bool pdl, cudaStream_t st);

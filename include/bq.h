@@ -189,6 +189,29 @@ bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, 
                   int64_t block_k, int dtype, const void* bias, void* out, int64_t ldo,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* bq_gemm restricted to the split-K decode kernel, with NO workspace argument
+ * and no device allocation: for callers that cannot allocate device memory
+ * where they call this -- a plugin inside another engine that owns every
+ * device byte, or a serving loop that plans all memory up front and forbids
+ * allocation (cudaMalloc can synchronise the device) once it is running.
+ * The kernel's scratch (64 KiB of arrival counters plus the split partials)
+ * is a fixed 16 MiB device array inside libbq, which every GPU that loads the
+ * library holds until the process exits.  Arguments and results are those of
+ * bq_gemm; the caller still provides inputs and output.  Limits: M <= 128,
+ * block_n = block_k = 128, 16-byte aligned operands and row strides, and a
+ * split-K plan whose scratch fits in 16 MiB (e.g. M = 64 with N = K = 4096
+ * fits; larger problems return BQ_ERR_UNSUPPORTED with the bytes needed).
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture.  Each call clears the counters
+ * it uses.  All calls share the one array, so calls that overlap on the GPU
+ * (different streams, or concurrent host threads) race and corrupt each
+ * other's results: serialise them.  The pages have no counterpart to this
+ * entry point; it exists for callers without an allocator. */
+bq_status bq_gemm_decode_noalloc(const void* qa, int64_t lda, const float* sa, const void* qw,
+                                 int64_t ldw, const float* sw, int64_t M, int64_t N, int64_t K,
+                                 int64_t block_n, int64_t block_k, int dtype, const void* bias,
+                                 void* out, int64_t ldo, void* stream);
+
 /* Workspace for bq_linear: bq_gemm's workspace (at offset 0, so the counter
  * rule above applies) followed by the activation codes and scales. */
 bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_n,

@@ -4,6 +4,7 @@
 // work, mirroring the block-wise INT8 page's ValueErrors (section 1: two-
 // dimensional block size, dynamic activations, int8-serialised checkpoint;
 // section 3: tensor-parallel block alignment), then chooses a kernel family.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -256,13 +257,17 @@ bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, 
                    workspace, workspace_bytes, stream, false);
 }
 
-// bq_linear workspace: [GEMM workspace (its counter region at offset 0)]
+// bq_linear workspace: [GEMM workspace, at least the 64 KiB counter region]
 // [activation codes M x ldq] [activation scales Kb x M].
 static void linear_layout(int64_t M, int64_t N, int64_t K, int64_t block_n, int64_t block_k,
                           int dtype, size_t* gemm_bytes, size_t* q_off, size_t* s_off,
                           size_t* total, int64_t* ldq) {
   *ldq = (int64_t)round_up((size_t)K, 16);
-  *gemm_bytes = round_up(bq::gemm_workspace_bytes(M, N, K, block_n, block_k, dtype), 256);
+  // the GEMM region always spans at least the counter region, so activation
+  // codes never land where a later decode call expects zeroed counters
+  *gemm_bytes = round_up(std::max(bq::gemm_workspace_bytes(M, N, K, block_n, block_k, dtype),
+                                  bq::kDecodeCounterBytes),
+                         256);
   *q_off = *gemm_bytes;
   *s_off = *q_off + round_up((size_t)(M * *ldq), 256);
   *total = *s_off + round_up((size_t)(cdiv(K, block_k) * M) * sizeof(float), 256);
@@ -298,7 +303,7 @@ bq_status bq_gemm_decode_noalloc(const void* qa, int64_t lda, const float* sa, c
                 plan.ws_bytes, bq::kNoAllocScratchBytes);
   void* scratch = nullptr;
   BQ_CHECK_CUDA(bq::noalloc_scratch(&scratch), "static scratch address");
-  if (plan.splits > 1) {
+  if (plan.ws_bytes > 0) {
     // arrival counters must start at zero; the partials need no clearing
     BQ_CHECK_CUDA(cudaMemsetAsync(scratch, 0, (size_t)plan.tiles * sizeof(unsigned),
                                   as_stream(stream)),

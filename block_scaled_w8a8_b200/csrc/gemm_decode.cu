@@ -13,9 +13,16 @@
 //    once); the grid has ~2 CTAs per SM so every SM keeps loads in flight;
 //  * per-K-block promotion in the epilogue warps (one weight row per thread,
 //    one token per TMEM column): acc[t] += P * sa[kb][t] * sw[tile][kb];
-//  * split partials go to a workspace; the last CTA to finish a tile sums
-//    them in split order (deterministic), adds the bias, writes bf16 and
-//    resets the tile's arrival counter.  The counters live in the first
+//  * cluster mode (enough weight tiles to fill the GPU): the S <= 8 split
+//    CTAs of a tile form a thread-block cluster; each leaves its fp32 partial
+//    in its own shared memory and, after a cluster barrier, reduces 128/S of
+//    the tile's rows by reading all S partials over distributed shared memory
+//    in split order (deterministic), adds the bias and writes bf16.  No
+//    global scratch is touched;
+//  * workspace mode (few tiles, so more splits than a cluster holds): split
+//    partials go to a workspace; the last CTA to finish a tile sums them in
+//    split order (deterministic), adds the bias, writes bf16 and resets the
+//    tile's arrival counter.  The counters live in the first
 //    kDecodeCounterBytes of the workspace (a fixed place, whatever the shape),
 //    so a workspace whose counter region starts zeroed stays usable by any
 //    sequence of calls; the partials after it need no initialisation;
@@ -50,6 +57,7 @@ struct DecParams {
   const float* sw;       // [Nb][Kb]
   int64_t M, N, K, Kb;
   int splits;
+  int cluster;           // 1: reduce over distributed shared memory
   const uint16_t* bias;
   uint16_t* out; int64_t ldo;
   float* part;           // [splits][M][N] (splits > 1)
@@ -72,6 +80,28 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 
 __device__ __forceinline__ void grid_dep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Four fp32 from CTA `rank`'s shared memory at the address matching `local`.
+__device__ __forceinline__ float4 ld_dsmem_f4(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(remote) : "memory");
+  return v;
 }
 
 template <int DT>
@@ -267,7 +297,14 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
     (void)ok;
     named_bar(1, 128);                 // all four epilogue warps decide together
-    if (!*abort_flag) {
+    if (p.cluster) {
+      // partial of this split -> own shared memory, [token][row]; the stage
+      // ring is free: every MMA has completed and consumed its loads
+      float* part_s = reinterpret_cast<float*>(smem);
+      const int row = 32 * q + lane;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) part_s[t * BN_W + row] = acc[t];
+    } else if (!*abort_flag) {
       const bool n_ok = n < p.N;
       if (p.splits == 1) {
         if (n_ok) {
@@ -304,6 +341,40 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
       }
     }
+  }
+
+  if (p.cluster) {
+    // every thread of every CTA in the cluster arrives: the partials are
+    // published, then each CTA reduces its share of rows in split order
+    cluster_sync_all();
+    const int S = p.splits;
+    const int rows_per = BN_W / S;             // 16, 32 or 64
+    const int quads = rows_per / 4;
+    const int c = (int)cluster_rank();
+    const float* part_s = reinterpret_cast<const float*>(smem);
+    const int items = (int)p.M * quads;
+    if (!*abort_flag) {
+      for (int it = threadIdx.x; it < items; it += kThreads) {
+        const int t = it / quads, qd = it - t * quads;
+        const int r0 = c * rows_per + 4 * qd;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < S; ++src) {
+          const float4 v = ld_dsmem_f4(part_s + t * BN_W + r0, (uint32_t)src);
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
+        const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t nn = (int64_t)tile * BN_W + r0 + j;
+          if (nn < p.N) {
+            const float b = p.bias ? bf16_bits_to_float(p.bias[nn]) : 0.f;
+            p.out[(int64_t)t * p.ldo + nn] = float_to_bf16_bits(vals[j] + b);
+          }
+        }
+      }
+    }
+    // keep this CTA's shared memory alive until every peer has read it
+    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -369,11 +440,13 @@ cudaError_t launch_nt(const GemmArgs& a, const DecodePlan& plan, void* ws, bool 
   p.sa = a.sa; p.sw = a.sw;
   p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK;
   p.splits = plan.splits;
+  p.cluster = plan.cluster ? 1 : 0;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  p.counters = plan.splits > 1 ? reinterpret_cast<unsigned*>(w) : nullptr;
-  p.part = plan.splits > 1 ? reinterpret_cast<float*>(w + kDecodeCounterBytes) : nullptr;
+  const bool use_ws = plan.splits > 1 && !plan.cluster;
+  p.counters = use_ws ? reinterpret_cast<unsigned*>(w) : nullptr;
+  p.part = use_ws ? reinterpret_cast<float*>(w + kDecodeCounterBytes) : nullptr;
   p.status = a.status;
 
   cudaLaunchConfig_t cfg = {};
@@ -381,11 +454,22 @@ cudaError_t launch_nt(const GemmArgs& a, const DecodePlan& plan, void* ws, bool 
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kTotal;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (plan.cluster) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = (unsigned)plan.splits;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kern, tW, tA, p);
 }
 
@@ -408,8 +492,22 @@ DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
   d.tiles = (N + BN_W - 1) / BN_W;
   const int64_t Kb = (K + BK - 1) / BK;
   // about two CTAs per SM, at most kMaxSplitKb K-blocks per split
-  int64_t s = std::max<int64_t>(1, (2 * 148 + d.tiles - 1) / d.tiles);
-  s = std::min<int64_t>(s, Kb);
+  const int64_t want = std::max<int64_t>(1, (2 * 148 + d.tiles - 1) / d.tiles);
+  d.cluster = false;
+  if (d.tiles >= 16) {
+    // cluster mode: a power-of-two split count <= 8 that leaves each split
+    // at least one K-block and at most kMaxSplitKb of them
+    int64_t s = 1;
+    while (s < 8 && s < want && 2 * s <= Kb) s *= 2;
+    if ((Kb + s - 1) / s <= kMaxSplitKb) {
+      d.splits = (int)s;
+      d.cluster = s > 1;
+      d.part_bytes = 0;
+      d.ws_bytes = 0;
+      return d;
+    }
+  }
+  int64_t s = std::min<int64_t>(want, Kb);
   s = std::max<int64_t>(s, (Kb + kMaxSplitKb - 1) / kMaxSplitKb);
   s = std::min<int64_t>(s, 65535);
   d.splits = (int)s;

@@ -17,8 +17,9 @@ struct DecodePlan {
   int nt;              // token tile (MMA N): 16, 32, 64 or 128
   int64_t tiles;       // 128-row weight tiles
   int splits;          // K splits per tile
+  bool cluster;        // splits reduce over distributed shared memory
   size_t part_bytes;   // fp32 split partials
-  size_t ws_bytes;     // counter region + partials (0 if splits == 1)
+  size_t ws_bytes;     // counter region + partials (0 unless workspace mode)
 };
 
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K);

@@ -217,13 +217,17 @@ def bench_decode(args, dist, bq, peaks, stream):
     gws = [bq.workspace(bq.gemm_workspace_size(M, N, K), dev) for M in Ms]
     torch.cuda.synchronize()
 
+    lws = bq.workspace(max(bq.linear_workspace_size(M, N, K) for M in Ms), dev)
+
     def step(phase, quant=True, gemm=True):
         def run():
             for j, M in enumerate(Ms):
                 wi = (4 * phase + j) % NW
-                if quant:
+                if quant and gemm:      # the public call: bq_linear
+                    bq.linear(xs[j], ws_q[wi], ws_s[wi], 128, 128, bq.INT8, out=outs[j], ws=lws)
+                elif quant:
                     bq.quant_act(xs[j], 128, bq.INT8, q=qa[j], s=sa[j])
-                if gemm:
+                else:
                     bq.gemm(qa[j], sa[j], ws_q[wi], ws_s[wi], 128, 128, bq.INT8, out=outs[j],
                             ws=gws[j])
         return run
@@ -246,7 +250,6 @@ def bench_decode(args, dist, bq, peaks, stream):
     hx = [x.cpu().pin_memory() for x in xs]
     ho = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in Ms]
     dx = [torch.empty_like(x, device=dev) for x in xs]
-    lws = bq.workspace(max(bq.linear_workspace_size(M, N, K) for M in Ms), dev)
 
     def e2e(phase):
         def run():

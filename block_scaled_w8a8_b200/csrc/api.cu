@@ -9,7 +9,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "../../include/bq.h"
+#include "bq.h"
 #include "bq_common.cuh"
 #include "bq_internal.h"
 #include "gemm_decode.h"

@@ -186,6 +186,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                     smem_u32(&full[i]));
       }
     }
+    // the next kernel in the stream may be scheduled now (it waits for this
+    // one before touching memory); then wait for the activation producer
+    if (lane == 0) asm volatile("griddepcontrol.launch_dependents;");
     grid_dep_wait();
     if (lane == 0) {
       for (int i = 0; i < first; ++i)
@@ -424,14 +427,68 @@ int num_sms() {
   return v > 0 ? v : 148;
 }
 
+// Largest number of clusters of `S` CTAs of this kernel the device can hold
+// at once (cached per device and S).
 template <int DT, int NT>
-cudaError_t launch_nt(const GemmArgs& a, const DecodePlan& plan, void* ws, bool pdl,
+int max_active_clusters(int S) {
+  static int cache[64][4] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int si = S == 2 ? 0 : S == 4 ? 1 : 2;
+  if (dev < 0 || dev >= 64) return 1;
+  if (cache[dev][si] == 0) {
+    using L = DSmem<NT>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, (unsigned)S, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kTotal;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = 1;
+    at.val.clusterDim.y = (unsigned)S;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_decode_kernel<DT, NT>, &cfg) != cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    cache[dev][si] = n;
+  }
+  return cache[dev][si];
+}
+
+// Split count for cluster mode: keep as many CTAs resident in the first wave
+// as possible (fewer waves first, then more resident CTAs, then larger S).
+template <int DT, int NT>
+int cluster_splits(int64_t tiles, int64_t Kb) {
+  int best = 2;
+  double best_score = -1.0;
+  for (int S = 8; S >= 2; S /= 2) {
+    if (S > Kb || (Kb + S - 1) / S > kMaxSplitKb) continue;
+    const int64_t n = max_active_clusters<DT, NT>(S);
+    const int64_t waves = (tiles + n - 1) / n;
+    const double score = (double)std::min<int64_t>(n, tiles) * S / (double)waves;
+    if (score > best_score) {
+      best_score = score;
+      best = S;
+    }
+  }
+  return best;
+}
+
+template <int DT, int NT>
+cudaError_t launch_nt(const GemmArgs& a, const DecodePlan& plan_in, void* ws, bool pdl,
                       cudaStream_t st) {
   using L = DSmem<NT>;
   auto kern = gemm_decode_kernel<DT, NT>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
   if (e != cudaSuccess) return e;
+  DecodePlan plan = plan_in;
+  if (plan.cluster) plan.splits = cluster_splits<DT, NT>(plan.tiles, (a.K + BK - 1) / BK);
   CUtensorMap tW, tA;
   if (!tmap(&tW, a.qw, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.ldw, BN_W) ||
       !tmap(&tA, a.qa, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.lda, NT))
@@ -494,18 +551,14 @@ DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
   // about two CTAs per SM, at most kMaxSplitKb K-blocks per split
   const int64_t want = std::max<int64_t>(1, (2 * 148 + d.tiles - 1) / d.tiles);
   d.cluster = false;
-  if (d.tiles >= 16) {
-    // cluster mode: a power-of-two split count <= 8 that leaves each split
-    // at least one K-block and at most kMaxSplitKb of them
-    int64_t s = 1;
-    while (s < 8 && s < want && 2 * s <= Kb) s *= 2;
-    if ((Kb + s - 1) / s <= kMaxSplitKb) {
-      d.splits = (int)s;
-      d.cluster = s > 1;
-      d.part_bytes = 0;
-      d.ws_bytes = 0;
-      return d;
-    }
+  if (d.tiles >= 16 && Kb >= 2 && (Kb + 7) / 8 <= kMaxSplitKb) {
+    // cluster mode: the split count (2, 4 or 8) is chosen at launch from the
+    // device's cluster occupancy; no workspace is needed
+    d.splits = 0;
+    d.cluster = true;
+    d.part_bytes = 0;
+    d.ws_bytes = 0;
+    return d;
   }
   int64_t s = std::min<int64_t>(want, Kb);
   s = std::max<int64_t>(s, (Kb + kMaxSplitKb - 1) / kMaxSplitKb);

@@ -16,7 +16,7 @@ constexpr size_t kDecodeCounterBytes = 65536;
 struct DecodePlan {
   int nt;              // token tile (MMA N): 16, 32, 64 or 128
   int64_t tiles;       // 128-row weight tiles
-  int splits;          // K splits per tile
+  int splits;          // K splits per tile (cluster mode: chosen at launch)
   bool cluster;        // splits reduce over distributed shared memory
   size_t part_bytes;   // fp32 split partials
   size_t ws_bytes;     // counter region + partials (0 unless workspace mode)

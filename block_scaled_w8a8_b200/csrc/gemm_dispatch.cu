@@ -7,7 +7,7 @@
 // the CUDA-core kernel.
 #include <cstdio>
 
-#include "../../include/bq.h"
+#include "bq.h"
 #include "gemm_paths.h"
 #include "gemm_decode.h"
 #include "gemm_tc.h"

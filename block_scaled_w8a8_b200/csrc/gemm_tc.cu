@@ -12,10 +12,16 @@
 //               partial P_kb (int32 for kind::i8, fp32 for kind::f8f6f4).
 //               Two TMEM buffers alternate so the MMA of block kb+1 overlaps
 //               the promotion of block kb.  Also owns the TMEM allocation.
-//   warps 4-7   epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
-//               per thread), promotes acc += P_kb * (sa[kb][m] * sw[nb][kb])
-//               in fp32 registers, frees the buffer, and after the last
-//               K-block adds the bias and stores bf16.
+//   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
+//               per thread) and columns [32*h, 32*h+32), h = (w-4)/4; it
+//               promotes acc += P_kb * (sa[kb][m] * sw[nb][kb]) in fp32
+//               registers with packed f32x2 arithmetic, frees the buffer, and
+//               after the last K-block adds the bias and stores bf16.
+// INT8 promotion without the int->float conversion unit: since
+// |P_kb| <= 128 * 128 * 128 < 2^22, the integer sum P_kb + 0x4B400000 (an
+// integer add on the ALU pipe) has the bits of the float 12582912 + P_kb
+// exactly, so one FADD recovers P_kb exactly and one FFMA promotes it (FMA
+// pipe, packed two per instruction).
 // A tile scheduler walks (expert, m-block, n-block) tiles; a dense problem is
 // one expert.  The grouped (MoE) problem reads its expert row ranges from
 // device memory, so no host read-back is needed.  Rows of a tile past the
@@ -42,7 +48,10 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BK = 128;
-constexpr int kThreads = 256;        // 8 warps: producer, MMA, 2 idle, 4 epilogue
+constexpr int kThreads = 640;        // 20 warps: producer, MMA, 2 idle, 16 epilogue
+constexpr int kEpiWarps = 16;
+constexpr uint32_t kMagicBits = 0x4B400000u;   // float 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;
 constexpr int kMaxE = 256;
 
 struct TcParams {
@@ -84,12 +93,6 @@ __device__ __forceinline__ void decode_tile(int t, const int* tp, const int* off
   nb = local / mblocks;
 }
 
-template <int DT>
-__device__ __forceinline__ float partial_to_float(uint32_t bits) {
-  if constexpr (DT == kInt8) return __int2float_rn((int)bits);
-  else return __uint_as_float(bits);
-}
-
 template <int DT, int BN, int S>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -121,7 +124,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 4);
+      mbar_init(smem_u32(&tempty[b]), kEpiWarps);
     }
     mbar_init(smem_u32(&drain[0]), 1);
     *abort_flag = 0;
@@ -241,62 +244,76 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else if (warp >= 4) {
     // ---------------- epilogue ----------------
+    constexpr int CW = 32;                         // columns per epilogue warp
     const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
     const int rit = 32 * q + lane;                 // row inside the tile
+    const uint32_t tcol = (uint32_t)(CW * half);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     uint32_t kcount = 0;
     int e_hint = 0;
     bool ok = true;
+    const uint64_t neg_magic2 = pack2(-kMagic, -kMagic);
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       int e, mb, nb;
       decode_tile(t, tp_s, off_s, E, p.nblk, e_hint, e, mb, nb);
       const int row0 = off_s[e] + mb * BM;
       const int64_t m = (int64_t)row0 + rit;
       const bool row_ok = rit < off_s[e + 1] - row0;
-      const int64_t n0 = (int64_t)nb * BN;
+      const int64_t n0 = (int64_t)nb * BN + CW * half;
       const float* sw_e = p.sw + (int64_t)e * p.sw_expert_stride;
-      float acc[BN];
+      const int64_t swrow = n0 < p.N ? wrow_block(n0, p.seam, p.N) * p.Kb : 0;
+      uint64_t acc[CW / 2];
 #pragma unroll
-      for (int i = 0; i < BN; ++i) acc[i] = 0.f;
-      float sa_next = row_ok ? p.sa[m] : 0.f;     // K-block 0
+      for (int i = 0; i < CW / 2; ++i) acc[i] = 0ull;
+      float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
+      float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
       for (int kb = 0; kb < p.Kb; ++kb) {
         const uint32_t buf = kcount & 1, tround = kcount >> 1;
-        const float sa_v = sa_next;
-        if (kb + 1 < p.Kb) sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
+        const float f = sa_next * sw_next;
+        if (kb + 1 < p.Kb) {
+          sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
+          sw_next = n0 < p.N ? __ldg(sw_e + swrow + kb + 1) : 0.f;
+        }
         if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x304u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          const int64_t nc = n0 + 32 * c;
-          const float swv = nc < p.N ? __ldg(sw_e + wrow_block(nc, p.seam, p.N) * p.Kb + kb) : 0.f;
-          const float f = sa_v * swv;
-          uint32_t r[32];
-          tmem_ld32(tmem_base + lane_base + buf * BN + 32 * c, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            acc[32 * c + i] = fmaf(partial_to_float<DT>(r[i]), f, acc[32 * c + i]);
-        }
+        uint32_t r[32];
+        const uint32_t taddr = tmem_base + lane_base + buf * BN + tcol;
+        tmem_ld32(taddr, r);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+        if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
+        const uint64_t f2 = pack2(f, f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          uint64_t x;
+          if constexpr (DT == kInt8) {
+            x = ((uint64_t)(r[2 * i + 1] + kMagicBits) << 32) | (uint64_t)(r[2 * i] + kMagicBits);
+            x = add2(x, neg_magic2);                             // exact P_kb
+          } else {
+            x = ((uint64_t)r[2 * i + 1] << 32) | (uint64_t)r[2 * i];
+          }
+          acc[i] = fma2(x, f2, acc[i]);
+        }
         ++kcount;
       }
       if (!ok) break;
-      if (row_ok) {
+      if (row_ok && n0 < p.N) {
         uint16_t* orow = p.out + m * p.ldo + n0;
-        const bool full_n = n0 + BN <= p.N;
+        const bool full_n = n0 + CW <= p.N;
         const bool vec = full_n && ((reinterpret_cast<uintptr_t>(orow) & 15) == 0);
         if (vec) {
 #pragma unroll
-          for (int j = 0; j < BN; j += 8) {
+          for (int j = 0; j < CW; j += 8) {
             uint32_t w[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              float v0 = acc[j + 2 * h], v1 = acc[j + 2 * h + 1];
+              float v0 = __uint_as_float((uint32_t)acc[j / 2 + h]);
+              float v1 = __uint_as_float((uint32_t)(acc[j / 2 + h] >> 32));
               if (p.bias) {
                 v0 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h));
                 v1 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h + 1));
@@ -307,11 +324,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < BN; ++j) {
+          for (int j = 0; j < CW; ++j) {
             if (n0 + j < p.N) {
-              float v = acc[j];
-              if (p.bias) v += bf16_bits_to_float(__ldg(p.bias + n0 + j));
-              orow[j] = float_to_bf16_bits(v);
+              float x = __uint_as_float((uint32_t)(acc[j / 2] >> (32 * (j & 1))));
+              if (p.bias) x += bf16_bits_to_float(__ldg(p.bias + n0 + j));
+              orow[j] = float_to_bf16_bits(x);
             }
           }
         }

@@ -92,9 +92,11 @@ quant_rows_kernel(const uint16_t* __restrict__ x, int64_t M_out, int64_t K, int6
                   const int32_t* __restrict__ perm, int64_t topk, int64_t gk, int64_t I_half,
                   uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ s,
                   uint16_t* __restrict__ h_out, bool vec_in, bool vec_out) {
-  // let a programmatically dependent GEMM start streaming its weights now; it
-  // waits (griddepcontrol.wait) before reading what this kernel writes
+  // Programmatic dependent launch: let the next kernel (a GEMM that streams
+  // its weights first) be scheduled now, then wait until the kernel before
+  // this one has finished and its writes are visible before touching memory.
   asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t Kb = (K + gk - 1) / gk;
   const int64_t n_groups = M_out * Kb;
@@ -197,13 +199,25 @@ cudaError_t launch_quant_act(const void* x, int64_t M_out, int64_t K, int64_t ld
   const int grid = grid_for_groups(M_out * Kb);
   auto xs = static_cast<const uint16_t*>(x);
   auto qs = static_cast<uint8_t*>(q);
+  // launched as a programmatic dependent of the preceding kernel: it waits on
+  // the GPU (griddepcontrol.wait) before reading or writing any memory, so
+  // only its launch latency overlaps the predecessor
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kWarpsPerCta * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
   if (dtype == kInt8)
-    quant_rows_kernel<kInt8, false><<<grid, kWarpsPerCta * 32, 0, st>>>(
-        xs, M_out, K, ldx, perm, topk, group_k, 0, qs, ldq, s, nullptr, vec_in, vec_out);
-  else
-    quant_rows_kernel<kFp8, false><<<grid, kWarpsPerCta * 32, 0, st>>>(
-        xs, M_out, K, ldx, perm, topk, group_k, 0, qs, ldq, s, nullptr, vec_in, vec_out);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, quant_rows_kernel<kInt8, false>, xs, M_out, K, ldx, perm,
+                              topk, group_k, (int64_t)0, qs, ldq, s, (uint16_t*)nullptr, vec_in,
+                              vec_out);
+  return cudaLaunchKernelEx(&cfg, quant_rows_kernel<kFp8, false>, xs, M_out, K, ldx, perm, topk,
+                            group_k, (int64_t)0, qs, ldq, s, (uint16_t*)nullptr, vec_in,
+                            vec_out);
 }
 
 cudaError_t launch_silu_mul_quant(const void* y, int64_t ldy, int64_t R, int64_t I,

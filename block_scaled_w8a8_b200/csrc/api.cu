@@ -94,7 +94,7 @@ const char* bq_status_string(int s) {
 const char* bq_last_error_message(void) { return g_msg; }
 
 bq_status bq_set_path(int path) {
-  BQ_CHECK_ARG(path >= BQ_PATH_AUTO && path <= BQ_PATH_DECODE, "unknown path %d", path);
+  BQ_CHECK_ARG(path >= BQ_PATH_AUTO && path <= BQ_PATH_GEMV, "unknown path %d", path);
   g_path = path;
   return ok();
 }

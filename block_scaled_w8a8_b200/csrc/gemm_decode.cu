@@ -48,7 +48,6 @@ using namespace sm100;
 
 constexpr int BN_W = 128;   // weight rows per tile (MMA M)
 constexpr int BK = 128;
-constexpr int kStages = 4;
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kMaxSplitKb = 32;  // K-blocks per split (their act scales sit in smem)
 
@@ -65,13 +64,20 @@ struct DecParams {
   unsigned* status;
 };
 
+// Ring depth per token tile: as deep as keeps a CTA under ~113 KB of shared
+// memory, so two CTAs fit on an SM (the next launch's CTAs can start while
+// this one finishes) and as many weight K-blocks as possible are in flight.
+template <int NT>
+constexpr int stages_for() { return NT <= 16 ? 6 : NT <= 32 ? 5 : NT <= 64 ? 4 : 3; }
+
 template <int NT>
 struct DSmem {
+  static constexpr int kStages = stages_for<NT>();
   static constexpr uint32_t kW = BN_W * BK, kA = NT * BK;
   static constexpr uint32_t kStage = kW + kA;
   static constexpr uint32_t kStages_ = kStages * kStage;
   static constexpr uint32_t kSa = kMaxSplitKb * NT * 4;
-  static constexpr uint32_t kTotal = 1024 + kStages_ + kSa + (2 * kStages + 5) * 8 + 16;
+  static constexpr uint32_t kTotal = 1024 + kStages_ + kSa + (2 * kStages + 17) * 8 + 16;
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -80,17 +86,6 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 
 __device__ __forceinline__ void grid_dep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-               ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
 }
 
 // Four fp32 from CTA `rank`'s shared memory at the address matching `local`.
@@ -110,21 +105,15 @@ __device__ __forceinline__ float pval(uint32_t b) {
   else return __uint_as_float(b);
 }
 
-// 32 lanes x 16 columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
+// TMEM buffers of NT columns (one K-block partial each): enough that the MMA
+// runs ahead of the epilogue instead of waiting for each buffer to drain.
+template <int NT>
+constexpr int tmem_bufs() { return NT <= 32 ? 8 : NT <= 64 ? 4 : 2; }
 
 template <int NT>
 constexpr uint32_t tmem_cols() {
-  return (2 * NT) <= 32 ? 32 : (2 * NT) <= 64 ? 64 : (2 * NT) <= 128 ? 128 : 256;
+  return (tmem_bufs<NT>() * NT) <= 32 ? 32 : (tmem_bufs<NT>() * NT) <= 64 ? 64
+       : (tmem_bufs<NT>() * NT) <= 128 ? 128 : 256;
 }
 
 template <int DT, int NT>
@@ -132,6 +121,7 @@ __global__ void __launch_bounds__(kThreads)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
                    const DecParams p) {
   using L = DSmem<NT>;
+  constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -139,10 +129,11 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStages_ + L::kSa);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
+  constexpr int kBufs = tmem_bufs<NT>();
   uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = bars + 2 * kStages + 2;
-  uint64_t* drain = bars + 2 * kStages + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* tempty = tfull + 8;
+  uint64_t* drain = tempty + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -157,7 +148,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
       mbar_init(smem_u32(&tempty[b]), 4);
     }
@@ -231,7 +222,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     for (int i = 0; i < nkb; ++i) {
       const int stage = i % kStages;
       const uint32_t phase = (uint32_t)((i / kStages) & 1);
-      const uint32_t buf = i & 1, tround = (uint32_t)(i >> 1);
+      const uint32_t buf = (uint32_t)(i % kBufs), tround = (uint32_t)(i / kBufs);
       if (!warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag, p.status, 0x402u) ||
           !warp_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x403u)) {
         ok = false;
@@ -276,7 +267,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
-      const uint32_t buf = i & 1, tround = (uint32_t)(i >> 1);
+      const uint32_t buf = (uint32_t)(i % kBufs), tround = (uint32_t)(i / kBufs);
       const float swv = __ldg(p.sw + (int64_t)tile * p.Kb + kb0 + i);
       if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x404u)) {
         ok = false;

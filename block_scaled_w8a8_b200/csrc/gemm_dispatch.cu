@@ -3,13 +3,17 @@
 //   SIMT     generic CUDA-core kernel: any shape, stride, block size.
 //   TCGEN05  TMA + tcgen05 kernel: block_n = block_k = 128, 16-byte strides.
 //   DECODE   swap-AB split-K weight-streaming tcgen05 kernel, M <= 128.
+//   GEMV     CUDA-core weight-streaming kernel, INT8, M <= 8 (forced only:
+//            measured on B200 it is no faster than DECODE at 1 token and
+//            slower at 8).
 // AUTO: M <= 128 -> DECODE, larger M -> TCGEN05, when they apply; otherwise
-// the CUDA-core kernel.
+// the generic CUDA-core kernel.
 #include <cstdio>
 
 #include "bq.h"
 #include "gemm_paths.h"
 #include "gemm_decode.h"
+#include "gemm_gemv.h"
 #include "gemm_tc.h"
 
 namespace bq {
@@ -34,8 +38,15 @@ static int run_simt(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
   return kRunOk;
 }
 
-static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
-  cudaError_t e = launch_gemm_tc(a, st);
+// kind: 0 = best tcgen05 kernel for the shape, 1 = 1-CTA, 2 = CTA pair.
+// The pair kernel's 256-row tiles pay off once there are more than 128 rows
+// (and for grouped problems, whose experts hold ~T*topk/E rows each).
+// Tile width of the CTA-pair kernel (128 or 256).
+static int g_pair_tile_n = 128;
+
+static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n, int kind = 0) {
+  const bool pair = kind == 2 || (kind == 0 && (a.offsets != nullptr || a.M > 128));
+  cudaError_t e = pair ? launch_gemm_tc_pair(a, g_pair_tile_n, st) : launch_gemm_tc(a, st);
   if (e != cudaSuccess) {
     snprintf(why, n, "tcgen05 GEMM launch: %s", cudaGetErrorString(e));
     return kRunCuda;
@@ -58,6 +69,15 @@ static int run_decode(const GemmArgs& a, void* ws, size_t ws_bytes, bool pdl, cu
   return kRunOk;
 }
 
+static int run_gemv(const GemmArgs& a, bool pdl, cudaStream_t st, char* why, size_t n) {
+  cudaError_t e = launch_gemm_gemv(a, pdl, st);
+  if (e != cudaSuccess) {
+    snprintf(why, n, "CUDA-core decode launch: %s", cudaGetErrorString(e));
+    return kRunCuda;
+  }
+  return kRunOk;
+}
+
 static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes, bool pdl,
                           cudaStream_t st, char* why, size_t why_len) {
   switch (path) {
@@ -69,11 +89,16 @@ static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes
     case BQ_PATH_DECODE:
       if (!decode_supported(a, why, why_len)) return kRunUnsupported;
       return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
+    case BQ_PATH_GEMV:
+      if (!gemv_supported(a, why, why_len)) return kRunUnsupported;
+      return run_gemv(a, pdl, st, why, why_len);
     case BQ_PATH_SIMT:
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
+    case BQ_PATH_TCGEN05_1CTA:
+    case BQ_PATH_TCGEN05_2CTA:
       if (!tc_supported(a, why, why_len)) return kRunUnsupported;
-      return run_tc(a, st, why, why_len);
+      return run_tc(a, st, why, why_len, path == BQ_PATH_TCGEN05 ? 0 : path - 3);
     default:
       snprintf(why, why_len, "kernel path %d is not available in this build", path);
       return kRunUnsupported;
@@ -101,8 +126,10 @@ int run_grouped_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cud
     case BQ_PATH_SIMT:
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
+    case BQ_PATH_TCGEN05_1CTA:
+    case BQ_PATH_TCGEN05_2CTA:
       if (!tc_supported(a, why, why_len)) return kRunUnsupported;
-      return run_tc(a, st, why, why_len);
+      return run_tc(a, st, why, why_len, path == BQ_PATH_TCGEN05 ? 0 : path - 3);
     default:
       snprintf(why, why_len, "kernel path %d is not available for grouped GEMM", path);
       return kRunUnsupported;

@@ -39,6 +39,7 @@
 #include "bq_common.cuh"
 #include "bq_internal.h"
 #include "gemm_tc.h"
+#include "gemm_tc_common.cuh"
 #include "sm100.cuh"
 
 namespace bq {
@@ -47,23 +48,19 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BK = 128;
+constexpr int BM = 128;
+using tc::BK;
+using tc::kMaxE;
+using tc::kMagic;
+using tc::kMagicBits;
+using tc::TcParams;
+using tc::decode_tile;
+using tc::wrow_block;
+using tc::make_tmap;
+using tc::sm_count;
+using tc::encode_fn;
 constexpr int kThreads = 640;        // 20 warps: producer, MMA, 2 idle, 16 epilogue
 constexpr int kEpiWarps = 16;
-constexpr uint32_t kMagicBits = 0x4B400000u;   // float 1.5 * 2^23
-constexpr float kMagic = 12582912.0f;
-constexpr int kMaxE = 256;
-
-struct TcParams {
-  const float* sa; int64_t sa_rows;
-  const float* sw; int64_t sw_expert_stride;
-  int64_t M, N, K, Kb, seam;
-  const int32_t* offsets; int E;
-  const uint16_t* bias;
-  uint16_t* out; int64_t ldo;
-  int nblk;
-  unsigned* status;
-};
 
 template <int BN, int S>
 struct Smem {
@@ -73,25 +70,6 @@ struct Smem {
   static constexpr uint32_t kMisc = 8 + 2 * (kMaxE + 1) * 4;
   static constexpr uint32_t kTotal = 1024 + kStages + kBars + kMisc;
 };
-
-__device__ __forceinline__ int64_t wrow_block(int64_t n, int64_t seam, int64_t N) {
-  if (seam <= 0 || seam >= N || n < seam) return n >> 7;
-  return ((seam + 127) >> 7) + ((n - seam) >> 7);
-}
-
-// Tile t -> (expert, m-block, n-block); m-blocks vary fastest so concurrent
-// CTAs share W tiles and the A operand of an expert stays in L2.
-__device__ __forceinline__ void decode_tile(int t, const int* tp, const int* off, int E, int nblk,
-                                            int& e_hint, int& e, int& mb, int& nb) {
-  int ee = e_hint;
-  while (ee + 1 < E && t >= tp[ee + 1]) ++ee;
-  e_hint = ee;
-  e = ee;
-  const int local = t - tp[ee];
-  const int mblocks = (off[ee + 1] - off[ee] + BM - 1) / BM;
-  mb = local % mblocks;
-  nb = local / mblocks;
-}
 
 template <int DT, int BN, int S>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -135,22 +113,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tma_prefetch_desc(&tmB);
   }
   // expert row ranges (sanitised: clamped to [0, M] and nondecreasing)
-  if (threadIdx.x == 32) {
-    int prev = 0;
-    bool bad = false;
-    for (int e = 0; e <= E; ++e) {
-      int v = p.offsets ? p.offsets[e] : (e == 0 ? 0 : (int)p.M);
-      if (e == 0 && v != 0) bad = true;
-      int c = min(max(v, prev), (int)p.M);
-      if (c != v) bad = true;
-      off_s[e] = (e == 0) ? 0 : c;
-      prev = off_s[e];
-    }
-    if (bad) record_status(p.status, kStatusBadInput, 0x201u);
-    tp_s[0] = 0;
-    for (int e = 0; e < E; ++e)
-      tp_s[e + 1] = tp_s[e] + ((off_s[e + 1] - off_s[e] + BM - 1) / BM) * p.nblk;
-  }
+  if (threadIdx.x == 32) tc::load_expert_ranges<BM>(p, off_s, tp_s);
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 2 * BN);
   tc_fence_before();
   __syncthreads();
@@ -169,7 +132,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       int e, mb, nb;
-      decode_tile(t, tp_s, off_s, E, p.nblk, e_hint, e, mb, nb);
+      decode_tile<BM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
       const int a_row = off_s[e] + mb * BM;
       const int b_row = e * (int)p.N + nb * BN;
       for (int kb = 0; kb < p.Kb; ++kb) {
@@ -256,7 +219,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint64_t neg_magic2 = pack2(-kMagic, -kMagic);
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       int e, mb, nb;
-      decode_tile(t, tp_s, off_s, E, p.nblk, e_hint, e, mb, nb);
+      decode_tile<BM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
       const int row0 = off_s[e] + mb * BM;
       const int64_t m = (int64_t)row0 + rit;
       const bool row_ok = rit < off_s[e + 1] - row0;
@@ -342,56 +305,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * BN);
   }
-}
-
-// ---- host side ------------------------------------------------------------------
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-// Row-major [rows, inner] uint8 tensor with row stride ld_bytes; box
-// [box_rows, 128 bytes], 128-byte swizzle, zero fill out of bounds.
-bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t ld_bytes,
-               uint32_t box_rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {ld_bytes};
-  cuuint32_t box[2] = {128u, box_rows};
-  cuuint32_t estr[2] = {1u, 1u};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int n[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return 148;
-  if (n[dev] == 0) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    n[dev] = v > 0 ? v : 148;
-  }
-  return n[dev];
 }
 
 template <int DT, int BN, int S>

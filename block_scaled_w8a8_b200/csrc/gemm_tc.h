@@ -10,6 +10,10 @@ namespace bq {
 
 // True if the tensor-core kernel can run this problem; otherwise writes why.
 bool tc_supported(const GemmArgs& a, char* why, size_t n);
+// Single-CTA kernel: 128 x 128 tiles.
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
+// CTA-pair kernel (cta_group::2): 256 x tile_n tiles (tile_n = 128 or 256);
+// same requirements.
+cudaError_t launch_gemm_tc_pair(const GemmArgs& a, int tile_n, cudaStream_t st);
 
 }  // namespace bq

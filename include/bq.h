@@ -83,7 +83,11 @@ typedef enum bq_path {
     BQ_PATH_AUTO = 0,     /* choose by shape and alignment */
     BQ_PATH_SIMT = 1,     /* generic CUDA-core kernel: any shape/stride */
     BQ_PATH_TCGEN05 = 2,  /* TMA + tcgen05 tensor-core kernel (large M) */
-    BQ_PATH_DECODE = 3    /* split-K weight-streaming kernel (small M) */
+    BQ_PATH_DECODE = 3,   /* split-K weight-streaming kernel (small M) */
+    BQ_PATH_TCGEN05_1CTA = 4,  /* force the 1-CTA 128x128-tile tcgen05 kernel */
+    BQ_PATH_TCGEN05_2CTA = 5,  /* force the CTA-pair 256x256-tile kernel */
+    BQ_PATH_GEMV = 6      /* CUDA-core weight-streaming kernel, INT8, M <= 8
+                             (forced only) */
 } bq_path;
 
 /* ---- library information and errors ---------------------------------- */

@@ -125,6 +125,7 @@ def test_quant_and_moe_argument_errors_on_host(L):
     assert L.bq_moe_combine(fake, 64, fake, fake, 4, 0, 64, fake, 64, None) == \
         bq.ERR_INVALID_ARG
     assert L.bq_set_path(9) == bq.ERR_INVALID_ARG
+    assert L.bq_set_path(7) == bq.ERR_INVALID_ARG
     assert L.bq_selftest_bounded_wait(0, None) == bq.ERR_INVALID_ARG
 
 

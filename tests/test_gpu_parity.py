@@ -133,11 +133,12 @@ TC_SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
 @pytest.mark.parametrize("dtype", [INT8, FP8])
 @pytest.mark.parametrize("M,N,K", TC_SHAPES)
-def test_gemm_tcgen05_vs_oracle(dtype, M, N, K):
+def test_gemm_tcgen05_vs_oracle(path, dtype, M, N, K):
     _, qa, sa, qw, sw, bb = make_problem(M, N, K, 128, 128, dtype, 300 + M, bias=(N % 256 == 0))
-    bq.set_path(bq.PATH_TCGEN05)
+    bq.set_path(path)
     out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, dtype,
                   bias=None if bb is None else dev_bf16(bb))
     torch.cuda.synchronize()
@@ -185,6 +186,33 @@ def test_gemm_decode_vs_oracle(dtype, M, N, K):
     ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bb)
     assert_gemm_close(out1, ref, f"decode dtype={dtype} {M}x{N}x{K}")
     assert torch.equal(out1, out2), "split-K reduction is not deterministic"
+
+
+GEMV_SHAPES = [(1, 640, 1008), (2, 4096, 4096), (8, 4096, 4096), (5, 1000, 4112),
+               (8, 384, 8192), (3, 130, 256), (7, 256, 16), (4, 200, 6144)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMV_SHAPES)
+def test_gemm_gemv_vs_oracle(M, N, K):
+    _, qa, sa, qw, sw, bb = make_problem(M, N, K, 128, 128, INT8, 700 + M, bias=(M % 2 == 0))
+    bq.set_path(bq.PATH_GEMV)
+    out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, INT8,
+                  bias=None if bb is None else dev_bf16(bb))
+    torch.cuda.synchronize()
+    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, INT8, bias_bf16=bb)
+    assert_gemm_close(out, ref, f"gemv {M}x{N}x{K}")
+
+
+def test_gemm_gemv_rejects_fp8_and_many_tokens():
+    bq.set_path(bq.PATH_GEMV)
+    _, qa, sa, qw, sw, _ = make_problem(9, 256, 256, 128, 128, INT8, 1)
+    with pytest.raises(bq.BqError) as ei:
+        bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, INT8)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+    _, qa, sa, qw, sw, _ = make_problem(4, 256, 256, 128, 128, FP8, 2)
+    with pytest.raises(bq.BqError) as ei:
+        bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, FP8)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("M", [1, 8, 64])
@@ -346,8 +374,9 @@ def test_moe_layer_stages_vs_oracle():
     assert (np.abs(ov - comb_ref) <= bf16_ulp(np.maximum(np.abs(ov), np.abs(comb_ref)))).all()
 
 
+@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
 @pytest.mark.parametrize("dtype", [INT8, FP8])
-def test_grouped_gemm_tcgen05_vs_oracle(dtype):
+def test_grouped_gemm_tcgen05_vs_oracle(path, dtype):
     p = moe_problem(T=300, H=384, I=256, E=8, dtype=dtype, seed=33)
     T, I, E, topk = p["T"], p["I"], p["E"], p["topk"]
     off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), E)
@@ -355,7 +384,7 @@ def test_grouped_gemm_tcgen05_vs_oracle(dtype):
     qa, sa = bq.moe_quant_gather(dev_bf16(p["x"]), perm, topk, 128, dtype)
     qx, sx = oracle.quant_act(p["x"], 128, dtype)
     rows = p_ref // topk
-    bq.set_path(bq.PATH_TCGEN05)
+    bq.set_path(path)
     y13 = bq.grouped_gemm(qa, sa, off, dev_u8(p["q13"]), dev_f32(p["s13"]), 128, 128,
                           n_seam=I, dtype=dtype)
     torch.cuda.synchronize()
@@ -365,7 +394,7 @@ def test_grouped_gemm_tcgen05_vs_oracle(dtype):
     assert_gemm_close(y13, ref13, "tcgen05 grouped w13")
 
 
-@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05])
+@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
 def test_grouped_gemm_leaves_rows_past_offsets_untouched(path):
     p = moe_problem(T=50, H=128, I=128, E=4)
     bq.set_path(path)

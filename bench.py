@@ -339,61 +339,90 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
             "dtype": "fp8_e4m3" if cfg.dtype else "int8"}
 
 
+class MoeLayer:
+    """The MoE layer of the block-int8 MoE workload (T tokens, E experts, top-k),
+    device-resident: routing, block-quantised w13 / w2, every intermediate,
+    and run(parts) that enqueues the layer's library calls in order.  The
+    full-size parity test drives the same object."""
+
+    PARTS = ("perm", "gather", "w13", "silu", "w2", "comb")
+
+    def __init__(self, bq, dev, cfg=None):
+        cfg = cfg or bq_synth.MOE
+        self.bq, self.cfg = bq, cfg
+        T, H, I, E, topk = cfg.T, cfg.H, cfg.I, cfg.E, cfg.topk
+        self.x = bq_synth.activations(T, H, cfg.seed, device=dev)
+        self.ids, self.tw = bq_synth.routing(T, E, topk, cfg.seed)
+        self.ids_d = torch.from_numpy(self.ids).to(dev)
+        self.tw_d = torch.from_numpy(self.tw).to(dev)
+        self.q13 = torch.empty(E, 2 * I, H, dtype=torch.uint8, device=dev)
+        self.s13 = torch.empty(E, 2 * cdiv(I, 128), cdiv(H, 128), dtype=torch.float32,
+                               device=dev)
+        self.q2 = torch.empty(E, H, I, dtype=torch.uint8, device=dev)
+        self.s2 = torch.empty(E, cdiv(H, 128), cdiv(I, 128), dtype=torch.float32, device=dev)
+        for e in range(E):
+            w13 = self.w13_fp32(e, dev)
+            for half in range(2):
+                q, s = bq.quant_weight(w13[half * I:(half + 1) * I].contiguous(), 128, 128,
+                                       cfg.dtype)
+                self.q13[e, half * I:(half + 1) * I] = q
+                self.s13[e, half * cdiv(I, 128):(half + 1) * cdiv(I, 128)] = s
+            del w13
+            q, s = bq.quant_weight(self.w2_fp32(e, dev), 128, 128, cfg.dtype)
+            self.q2[e], self.s2[e] = q, s
+        R = T * topk
+        self.off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.perm = torch.empty(R, dtype=torch.int32, device=dev)
+        self.inv = torch.empty(R, dtype=torch.int32, device=dev)
+        self.qa = torch.empty(R, H, dtype=torch.uint8, device=dev)
+        self.sa = torch.empty(cdiv(H, 128), R, dtype=torch.float32, device=dev)
+        self.y13 = torch.empty(R, 2 * I, dtype=torch.bfloat16, device=dev)
+        self.qh = torch.empty(R, I, dtype=torch.uint8, device=dev)
+        self.sh = torch.empty(cdiv(I, 128), R, dtype=torch.float32, device=dev)
+        self.y2 = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.ws = bq.workspace(bq.grouped_gemm_workspace_size(R, 2 * I, H, E), dev)
+        torch.cuda.synchronize()
+
+    def w13_fp32(self, e, dev):
+        c = self.cfg
+        return bq_synth.weights(2 * c.I, c.H, c.w_std, c.seed + 31 * e, device=dev)
+
+    def w2_fp32(self, e, dev):
+        c = self.cfg
+        return bq_synth.weights(c.H, c.I, c.w_std, c.seed + 31 * e + 1, device=dev)
+
+    def run(self, parts=PARTS):
+        bq, c = self.bq, self.cfg
+        L = bq.lib()
+        st = torch.cuda.current_stream().cuda_stream
+        if "perm" in parts:
+            bq._check(L.bq_moe_permute(self.ids_d.data_ptr(), c.T, c.topk, c.E,
+                                       self.off.data_ptr(), self.perm.data_ptr(),
+                                       self.inv.data_ptr(), None, 0, st))
+        if "gather" in parts:
+            bq.moe_quant_gather(self.x, self.perm, c.topk, 128, c.dtype, q=self.qa, s=self.sa)
+        if "w13" in parts:
+            bq.grouped_gemm(self.qa, self.sa, self.off, self.q13, self.s13, 128, 128, c.I,
+                            c.dtype, out=self.y13, ws=self.ws)
+        if "silu" in parts:
+            bq.moe_silu_mul_quant(self.y13, c.I, 128, c.dtype, q=self.qh, s=self.sh)
+        if "w2" in parts:
+            bq.grouped_gemm(self.qh, self.sh, self.off, self.q2, self.s2, 128, 128, 0, c.dtype,
+                            out=self.y2, ws=self.ws)
+        if "comb" in parts:
+            bq.moe_combine(self.y2, self.inv, self.tw_d, out=self.out)
+
+
 def bench_moe(args, dist, bq, peaks, stream):
     cfg = bq_synth.MOE
     dev = torch.device("cuda", torch.cuda.current_device())
     T, H, I, E, topk = cfg.T, cfg.H, cfg.I, cfg.E, cfg.topk
-    x = bq_synth.activations(T, H, cfg.seed, device=dev)
-    ids, tw = bq_synth.routing(T, E, topk, cfg.seed)
-    ids_d = torch.from_numpy(ids).to(dev)
-    tw_d = torch.from_numpy(tw).to(dev)
-    q13 = torch.empty(E, 2 * I, H, dtype=torch.uint8, device=dev)
-    s13 = torch.empty(E, 2 * cdiv(I, 128), cdiv(H, 128), dtype=torch.float32, device=dev)
-    q2 = torch.empty(E, H, I, dtype=torch.uint8, device=dev)
-    s2 = torch.empty(E, cdiv(H, 128), cdiv(I, 128), dtype=torch.float32, device=dev)
-    for e in range(E):
-        w13 = bq_synth.weights(2 * I, H, cfg.w_std, cfg.seed + 31 * e, device=dev)
-        for half in range(2):
-            q, s = bq.quant_weight(w13[half * I:(half + 1) * I].contiguous(), 128, 128, cfg.dtype)
-            q13[e, half * I:(half + 1) * I] = q
-            s13[e, half * cdiv(I, 128):(half + 1) * cdiv(I, 128)] = s
-        del w13
-        w2 = bq_synth.weights(H, I, cfg.w_std, cfg.seed + 31 * e + 1, device=dev)
-        q, s = bq.quant_weight(w2, 128, 128, cfg.dtype)
-        q2[e], s2[e] = q, s
-        del w2
     R = T * topk
-    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(R, dtype=torch.int32, device=dev)
-    inv = torch.empty(R, dtype=torch.int32, device=dev)
-    qa = torch.empty(R, H, dtype=torch.uint8, device=dev)
-    sa = torch.empty(cdiv(H, 128), R, dtype=torch.float32, device=dev)
-    y13 = torch.empty(R, 2 * I, dtype=torch.bfloat16, device=dev)
-    qh = torch.empty(R, I, dtype=torch.uint8, device=dev)
-    sh = torch.empty(cdiv(I, 128), R, dtype=torch.float32, device=dev)
-    y2 = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
-    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-    ws13 = bq.workspace(bq.grouped_gemm_workspace_size(R, 2 * I, H, E), dev)
-    torch.cuda.synchronize()
-    L = bq.lib()
-    st = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+    moe = MoeLayer(bq, dev, cfg)
 
-    def layer(parts=("perm", "gather", "w13", "silu", "w2", "comb")):
-        def run():
-            if "perm" in parts:
-                bq._check(L.bq_moe_permute(ids_d.data_ptr(), T, topk, E, off.data_ptr(),
-                                           perm.data_ptr(), inv.data_ptr(), None, 0, st()))
-            if "gather" in parts:
-                bq.moe_quant_gather(x, perm, topk, 128, cfg.dtype, q=qa, s=sa)
-            if "w13" in parts:
-                bq.grouped_gemm(qa, sa, off, q13, s13, 128, 128, I, cfg.dtype, out=y13, ws=ws13)
-            if "silu" in parts:
-                bq.moe_silu_mul_quant(y13, I, 128, cfg.dtype, q=qh, s=sh)
-            if "w2" in parts:
-                bq.grouped_gemm(qh, sh, off, q2, s2, 128, 128, 0, cfg.dtype, out=y2, ws=ws13)
-            if "comb" in parts:
-                bq.moe_combine(y2, inv, tw_d, out=out)
-        return run
+    def layer(parts=MoeLayer.PARTS):
+        return lambda: moe.run(parts)
 
     g = [capture(layer(), stream)]
     gg = [capture(layer(("w13", "w2")), stream)]
@@ -420,36 +449,44 @@ def bench_moe(args, dist, bq, peaks, stream):
 # CPU oracle (baseline leg and reference arm)
 # --------------------------------------------------------------------------
 
-def oracle_decode_sample(n_rows: int):
-    """One decode step restricted to the first n_rows weight rows: the oracle's
-    activation quantisation for M in {1,8,32,64} and its GEMM against an
-    [n_rows, 4096] weight slice.  Returns (seconds, algorithmic bytes)."""
-    import oracle
-    K = 4096
-    w = bq_synth.weights(n_rows, K, 0.02, 100).numpy()
-    qw, sw = oracle.quant_weight(w, 128, 128, oracle.INT8)
-    xs = [bq_synth.bf16_bits(bq_synth.activations(M, K, c.seed, c.n_outliers,
-                                                  c.outlier_scale))
-          for M, c in zip(bq_synth.DECODE_MS, bq_synth.DECODE)]
-    t0 = time.perf_counter()
-    for xb in xs:
-        qa, sa = oracle.quant_act(xb, 128, oracle.INT8)
-        oracle.gemm(qa, sa, qw, sw, 128, 128, oracle.INT8)
-    dt = time.perf_counter() - t0
-    Nb, Kb = cdiv(n_rows, 128), K // 128
-    nbytes = sum(n_rows * K + 4 * Nb * Kb + 2 * M * K + 2 * M * n_rows
-                 for M in bq_synth.DECODE_MS)
-    return dt, nbytes
+class OracleDecode:
+    """The decode workload on the CPU oracle: activation quantisation for
+    M in {1, 8, 32, 64} and the block-scaled GEMM against the 4096 x 4096 INT8
+    weight (the first of the GPU leg's rotating weights).  Inputs are prepared
+    once; step() runs one whole decode step and returns its seconds."""
+
+    def __init__(self, n_rows: int = 4096):
+        import oracle
+        self.oracle = oracle
+        K = 4096
+        w = bq_synth.weights(n_rows, K, 0.02, 100).numpy()
+        self.qw, self.sw = oracle.quant_weight(w, 128, 128, oracle.INT8)
+        self.xs = [bq_synth.bf16_bits(bq_synth.activations(M, K, c.seed, c.n_outliers,
+                                                           c.outlier_scale))
+                   for M, c in zip(bq_synth.DECODE_MS, bq_synth.DECODE)]
+        Nb, Kb = cdiv(n_rows, 128), K // 128
+        self.n_rows = n_rows
+        self.bytes_per_step = sum(n_rows * K + 4 * Nb * Kb + 2 * M * K + 2 * M * n_rows
+                                  for M in bq_synth.DECODE_MS)
+
+    def step(self) -> float:
+        o = self.oracle
+        t0 = time.perf_counter()
+        for xb in self.xs:
+            qa, sa = o.quant_act(xb, 128, o.INT8)
+            o.gemm(qa, sa, self.qw, self.sw, 128, 128, o.INT8)
+        return time.perf_counter() - t0
 
 
-def cpu_baseline(seconds_target=20.0):
-    dt, nb = oracle_decode_sample(256)
-    rows = int(min(4096, max(128, 256 * seconds_target / max(dt, 1e-3) / 2)))
-    rows = max(128, rows // 128 * 128)
-    dt, nb = oracle_decode_sample(rows)
-    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"one decode step (M in 1,8,32,64; K=4096) on the first {rows} of the "
-                      f"4096 weight rows; single-threaded C oracle; {dt:.1f} s"}
+def cpu_baseline(seconds_target=15.0):
+    od = OracleDecode()
+    first = od.step()
+    reps = max(1, int(seconds_target / max(first, 1e-3)))
+    dt = sum(od.step() for _ in range(reps))
+    return {"value": reps * od.bytes_per_step / dt / 1e9, "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{reps} whole decode steps (M in 1,8,32,64; N = K = 4096) after one "
+                      f"untimed step; single-threaded C oracle; {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -457,24 +494,21 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = 256
+    od = OracleDecode()
     for _ in range(args.warmup):
-        oracle_decode_sample(rows)
-    tot_t, tot_b = 0.0, 0
-    for _ in range(args.steps):
-        dt, nb = oracle_decode_sample(rows)
-        tot_t += dt
-        tot_b += nb
-    v = tot_b / tot_t / 1e9
+        od.step()
+    tot_t = sum(od.step() for _ in range(args.steps))
+    v = args.steps * od.bytes_per_step / tot_t / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": "decode_int8_n4096_k4096_m1-8-32-64",
-                       "sample_rows": rows, "world_size": world},
+                       "M": list(bq_synth.DECODE_MS), "N": 4096, "K": 4096,
+                       "block": [128, 128], "world_size": world},
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"each step: one decode step on {rows} of 4096 weight "
-                                       "rows, single-threaded C oracle"},
+                             "sample": "each step: one whole decode step (M in 1,8,32,64; "
+                                       "N = K = 4096), single-threaded C oracle"},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

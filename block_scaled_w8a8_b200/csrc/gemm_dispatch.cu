@@ -38,14 +38,14 @@ static int run_simt(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
   return kRunOk;
 }
 
-// kind: 0 = best tcgen05 kernel for the shape, 1 = 1-CTA, 2 = CTA pair.
-// The pair kernel's 256-row tiles pay off once there are more than 128 rows
-// (and for grouped problems, whose experts hold ~T*topk/E rows each).
-// Tile width of the CTA-pair kernel (128 or 256).
-static int g_pair_tile_n = 128;
+// kind: 0 = default tcgen05 kernel, 1 = 1-CTA, 2 = CTA pair.  Measured on
+// B200 the CTA-pair kernel is slower than the 1-CTA kernel for every workload
+// here (its epilogue drains TMEM more slowly), so it runs only when forced.
+// Tile width of the CTA-pair kernel (128 or 256; 256 measured faster).
+static int g_pair_tile_n = 256;
 
 static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n, int kind = 0) {
-  const bool pair = kind == 2 || (kind == 0 && (a.offsets != nullptr || a.M > 128));
+  const bool pair = kind == 2;
   cudaError_t e = pair ? launch_gemm_tc_pair(a, g_pair_tile_n, st) : launch_gemm_tc(a, st);
   if (e != cudaSuccess) {
     snprintf(why, n, "tcgen05 GEMM launch: %s", cudaGetErrorString(e));

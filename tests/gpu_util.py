@@ -76,3 +76,27 @@ def assert_scales_equal(s_gpu_kbmajor: torch.Tensor, s_ref_rowmajor: np.ndarray,
         i = tuple(idx[0])
         raise AssertionError(f"{what}: {len(idx)} scales differ; first at {i}: "
                              f"gpu {sg[i]!r} oracle {s_ref_rowmajor[i]!r}")
+
+
+def assert_combine_close(out: torch.Tensor, ref_bits: np.ndarray, y_bits: np.ndarray,
+                         inv_perm: np.ndarray, w: np.ndarray, what: str = "combine"):
+    """The weighted top-k combine is an fp32 sum of fp32 products rounded once
+    to bf16; the oracle's is exact before its one rounding.  Where the terms
+    nearly cancel, the kernel's fp32 product roundings (each within 2^-24 of
+    its term) exceed one bf16 ulp of the small result, so the bound is one
+    bf16 ulp plus 2^-22 * sum_j |w_j * y_j| (a factor-4 margin over the two
+    fp32 roundings)."""
+    import oracle
+    g = bf16_values(out)
+    r = oracle.bf16_to_f64(ref_bits)
+    T, topk = w.shape
+    yv = oracle.bf16_to_f64(y_bits)
+    mag = np.zeros_like(r)
+    for j in range(topk):
+        mag += np.abs(w[:, j:j + 1].astype(np.float64) * yv[inv_perm.reshape(T, topk)[:, j]])
+    tol = bf16_ulp(np.maximum(np.abs(g), np.abs(r))) + 2.0 ** -22 * mag
+    bad = np.abs(g - r) > tol
+    if bad.any():
+        i = tuple(np.argwhere(bad)[0])
+        raise AssertionError(f"{what}: {int(bad.sum())} outputs beyond the fp32-sum bound; "
+                             f"first at {i}: gpu {g[i]!r} oracle {r[i]!r} tol {tol[i]!r}")

@@ -11,7 +11,8 @@ import torch
 import block_scaled_w8a8_b200 as bq
 import bq_synth
 import oracle
-from gpu_util import (assert_codes_equal, assert_gemm_close, assert_scales_equal, bf16_ulp,
+from gpu_util import (assert_codes_equal, assert_combine_close, assert_gemm_close,
+                      assert_scales_equal, bf16_ulp,
                       bf16_values, dev_bf16, dev_f32, dev_i32, dev_u8, host_bits)
 
 pytestmark = pytest.mark.gpu
@@ -369,9 +370,8 @@ def test_moe_layer_stages_vs_oracle():
     # combine: fp32 accumulate, one rounding
     out = bq.moe_combine(y2, inv, dev_f32(p["tw"]))
     torch.cuda.synchronize()
-    comb_ref = oracle.bf16_to_f64(oracle.moe_combine(host_bits(y2), i_ref, p["tw"]))
-    ov = bf16_values(out)
-    assert (np.abs(ov - comb_ref) <= bf16_ulp(np.maximum(np.abs(ov), np.abs(comb_ref)))).all()
+    yb = host_bits(y2)
+    assert_combine_close(out, oracle.moe_combine(yb, i_ref, p["tw"]), yb, i_ref, p["tw"])
 
 
 @pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])

@@ -3,22 +3,29 @@
 // Same contraction as the other GEMMs (block-wise INT8 page, sections 2 and 4;
 // blockwise FP8 of the SGLang quantization doc), for M <= 128 tokens and
 // block_n = block_k = 128.  With so few tokens the layer is bound by reading
-// the weights once from HBM, so the kernel is organised around that stream:
+// the weights once from HBM, so the kernel is organised around that stream
+// and around what must wait for the preceding kernel:
 //
 //  * swap-AB: the 128 weight rows of a tile are the MMA's M dimension and the
 //    tokens (padded to NT = 16/32/64/128) its N dimension, so no MMA rows are
 //    wasted on padding tokens;  D[n, t] = sum_k W[n, k] * A[t, k];
 //  * split-K: CTA (tile, split) streams the K-blocks [kb0, kb1) of one 128-row
-//    weight tile through a TMA ring (16 KB per K-block, all loads in flight at
-//    once); the grid has ~2 CTAs per SM so every SM keeps loads in flight;
+//    weight tile through a TMA ring, small enough that two CTAs share an SM;
+//  * before griddepcontrol.wait (programmatic dependent launch) a CTA issues
+//    its first weight stages and reads its weight scales: neither depends on
+//    the preceding kernel, so both overlap that kernel's tail.  The next
+//    kernel is released once this CTA's first activation tile has arrived,
+//    so its weight stream does not queue ahead of this CTA's activation reads;
 //  * per-K-block promotion in the epilogue warps (one weight row per thread,
-//    one token per TMEM column): acc[t] += P * sa[kb][t] * sw[tile][kb];
+//    one token per TMEM column), each K-block drained as soon as its MMAs
+//    complete: acc[t] += P * sa[kb][t] * sw[tile][kb];
 //  * cluster mode (enough weight tiles to fill the GPU): the S <= 8 split
-//    CTAs of a tile form a thread-block cluster; each leaves its fp32 partial
-//    in its own shared memory and, after a cluster barrier, reduces 128/S of
-//    the tile's rows by reading all S partials over distributed shared memory
-//    in split order (deterministic), adds the bias and writes bf16.  No
-//    global scratch is touched;
+//    CTAs of a tile form a thread-block cluster.  Each pushes the partial of
+//    every row to the CTA that owns the row (128/S rows each) over
+//    distributed shared memory and arrives on that CTA's mbarrier; the owner
+//    sums the S partials in split order (deterministic), adds the bias and
+//    writes bf16.  One cluster barrier, at start-up, makes the peers'
+//    mbarriers visible; no global scratch is touched;
 //  * workspace mode (few tiles, so more splits than a cluster holds): split
 //    partials go to a workspace; the last CTA to finish a tile sums them in
 //    split order (deterministic), adds the bias, writes bf16 and resets the
@@ -26,9 +33,8 @@
 //    kDecodeCounterBytes of the workspace (a fixed place, whatever the shape),
 //    so a workspace whose counter region starts zeroed stays usable by any
 //    sequence of calls; the partials after it need no initialisation;
-//  * programmatic dependent launch: the weight loads are issued before
-//    griddepcontrol.wait, so they overlap the activation quantiser that
-//    produces this kernel's A operand.
+//  * TMEM is released as soon as the epilogue has read it, so the CTA's exit
+//    (which releases the next kernel) is not held up.
 #include <cuda.h>
 
 #include <algorithm>
@@ -64,39 +70,44 @@ struct DecParams {
   unsigned* status;
 };
 
-// Ring depth per token tile: as deep as keeps a CTA under ~113 KB of shared
-// memory, so two CTAs fit on an SM (the next launch's CTAs can start while
-// this one finishes) and as many weight K-blocks as possible are in flight.
-template <int NT>
-constexpr int stages_for() { return NT <= 16 ? 6 : NT <= 32 ? 5 : NT <= 64 ? 4 : 3; }
-
+// Shared memory of one CTA.  The ring is as deep as keeps the CTA within
+// ~112 KB (two CTAs per SM, so the next launch's CTAs can start streaming
+// while this one finishes); NT = 128 takes one CTA per SM.
 template <int NT>
 struct DSmem {
-  static constexpr int kStages = stages_for<NT>();
-  static constexpr uint32_t kW = BN_W * BK, kA = NT * BK;
+  static constexpr uint32_t kW = BN_W * BK;                 // weight stage
+  static constexpr uint32_t kA = NT * BK;                   // activation tile
   static constexpr uint32_t kStage = kW + kA;
-  static constexpr uint32_t kStages_ = kStages * kStage;
   static constexpr uint32_t kSa = kMaxSplitKb * NT * 4;
-  static constexpr uint32_t kTotal = 1024 + kStages_ + kSa + (2 * kStages + 17) * 8 + 16;
+  static constexpr uint32_t kSw = kMaxSplitKb * 4;
+  static constexpr int kNtp = NT + 4;                        // padded token row (floats)
+  static constexpr uint32_t kSlots = kNtp * BN_W * 4;        // [S][128/S][kNtp] fp32
+  static constexpr uint32_t kBars = 64 * 8;
+  static constexpr uint32_t kFixed = 1024 + kSa + kSw + kSlots + kBars;
+  static constexpr uint32_t kBudget = NT <= 64 ? 112u * 1024u : 200u * 1024u;
+  static constexpr int kStagesRaw = (int)((kBudget - kFixed) / kStage);
+  static constexpr int kStages = kStagesRaw < 2 ? 2 : kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr uint32_t kRing = kStages * kStage;
+  // offsets from the 1024-aligned base
+  static constexpr uint32_t oSa = kRing;
+  static constexpr uint32_t oSw = oSa + kSa;
+  static constexpr uint32_t oSlots = oSw + kSw;
+  static constexpr uint32_t oBars = oSlots + kSlots;
+  static constexpr uint32_t kTotal = 1024 + oBars + kBars;
+  static_assert(kRing % 1024 == 0 && kStage % 1024 == 0, "MMA operand tiles need 1 KB alignment");
+  static_assert(kTotal <= 227u * 1024u, "shared memory budget");
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// Four fp32 from CTA `rank`'s shared memory at the address matching `local`.
-__device__ __forceinline__ float4 ld_dsmem_f4(const float* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-               : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(remote) : "memory");
-  return v;
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 template <int DT>
@@ -116,32 +127,64 @@ constexpr uint32_t tmem_cols() {
        : (tmem_bufs<NT>() * NT) <= 128 ? 128 : 256;
 }
 
+// Bounded wait on a local mbarrier whose arrivals come from other CTAs of the
+// cluster (acquire at cluster scope).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort_flag, unsigned* status,
+                                                  unsigned site) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 63u) == 63u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitTimeoutNs) {
+        record_status(status, kStatusTimeout, site);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 template <int DT, int NT>
 __global__ void __launch_bounds__(kThreads)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
                    const DecParams p) {
   using L = DSmem<NT>;
   constexpr int kStages = L::kStages;
+  constexpr int kBufs = tmem_bufs<NT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* sa_s = reinterpret_cast<float*>(smem + L::kStages_);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStages_ + L::kSa);
+  float* sa_s = reinterpret_cast<float*>(smem + L::oSa);
+  float* sw_s = reinterpret_cast<float*>(smem + L::oSw);
+  float* slots = reinterpret_cast<float*>(smem + L::oSlots);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::oBars);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  constexpr int kBufs = tmem_bufs<NT>();
-  uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = tfull + 8;
-  uint64_t* drain = tempty + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* empty = bars + 8;
+  uint64_t* tfull = bars + 16;
+  uint64_t* tempty = bars + 24;
+  uint64_t* drain = bars + 32;
+  uint64_t* red = bars + 33;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 34);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* epi_abort = reinterpret_cast<volatile int*>(tmem_slot + 3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, split = blockIdx.y;
   const int kb0 = (int)((int64_t)split * p.Kb / p.splits);
   const int kb1 = (int)((int64_t)(split + 1) * p.Kb / p.splits);
   const int nkb = kb1 - kb0;
+  const int first = min(nkb, kStages);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -153,10 +196,26 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
       mbar_init(smem_u32(&tempty[b]), 4);
     }
     mbar_init(smem_u32(&drain[0]), 1);
+    mbar_init(smem_u32(&red[0]), BN_W);     // one arrival per pushed row
     *abort_flag = 0;
     fence_mbar_init();
+    // The weights do not depend on the preceding kernel: the first stages are
+    // requested before this CTA waits for its activations.
+    tma_prefetch_desc(&tmW);
+    for (int i = 0; i < first; ++i) {
+      mbar_arrive_expect_tx(smem_u32(&full[i]), L::kStage);
+      tma_load_2d(smem_u32(smem + i * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
+                  smem_u32(&full[i]));
+    }
+    tma_prefetch_desc(&tmA);
   }
+  // this split's weight scales: constant data, read before the wait
+  if (threadIdx.x >= 64 && threadIdx.x - 64 < nkb)
+    sw_s[threadIdx.x - 64] = __ldg(p.sw + (int64_t)tile * p.Kb + kb0 + (threadIdx.x - 64));
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), tmem_cols<NT>());
+  // start-up cluster barrier: the peers' mbarriers are initialised before
+  // anyone arrives on them remotely (waited on just before the push)
+  if (p.cluster) cluster_arrive();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -164,23 +223,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      tma_prefetch_desc(&tmW);
-      tma_prefetch_desc(&tmA);
-    }
-    // weights first (independent of the preceding kernel), then activations
-    const int first = min(nkb, kStages);
-    if (lane == 0) {
-      for (int i = 0; i < first; ++i) {
-        mbar_arrive_expect_tx(smem_u32(&full[i]), L::kStage);
-        tma_load_2d(smem_u32(smem + i * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
-                    smem_u32(&full[i]));
-      }
-    }
-    // the next kernel in the stream may be scheduled now (it waits for this
-    // one before touching memory); then wait for the activation producer
-    if (lane == 0) asm volatile("griddepcontrol.launch_dependents;");
-    grid_dep_wait();
+    grid_dep_wait();                              // the activation codes are ready
     if (lane == 0) {
       for (int i = 0; i < first; ++i)
         tma_load_2d(smem_u32(smem + i * L::kStage + L::kW), &tmA, (kb0 + i) * BK, 0,
@@ -215,6 +258,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t idesc = instr_desc<DT>(BN_W, NT);
@@ -229,6 +273,10 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         break;
       }
       tc_fence_after();
+      // the first activation tile has arrived: this CTA's reads of the
+      // preceding kernel's output are under way, so the next kernel may be
+      // scheduled (earlier, its weight stream would queue ahead of them)
+      if (i == 0 && lane == 0) asm volatile("griddepcontrol.launch_dependents;");
       if (lane == 0) {
         const uint32_t d = tmem_base + buf * NT;
         const uint64_t a0 = smem_desc_k128(smem_u32(smem + stage * L::kStage));
@@ -242,14 +290,20 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
       __syncwarp();
       issued_any = true;
     }
-    if (!ok && issued_any) {
-      // wait (bounded) for the MMAs already issued before TMEM is freed
+    (void)ok;
+    if (issued_any) {
+      // every MMA issued has completed (bounded wait) before TMEM is freed
       if (lane == 0) mma_commit(smem_u32(&drain[0]));
       __syncwarp();
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(smem_u32(&drain[0]), 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
+    // free TMEM once the epilogue warps have read their last partial
+    named_bar(2, 160);
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols<NT>());
+    __syncwarp();
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;                       // TMEM lane quadrant of this warp
@@ -265,40 +319,117 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+    // each K-block is drained as soon as its MMAs complete (waiting for more
+    // K-blocks first only delays the last ones), up to 64 columns per wait
+    constexpr int kCk = NT / 16;                  // 16-column chunks per K-block
+    constexpr int kCkB = kCk > 4 ? 4 : kCk;       // chunks per wait
+    constexpr int kHalves = kCk / kCkB;           // waits per K-block
+    constexpr int kKbPer = 1;
     bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
-      const uint32_t buf = (uint32_t)(i % kBufs), tround = (uint32_t)(i / kBufs);
-      const float swv = __ldg(p.sw + (int64_t)tile * p.Kb + kb0 + i);
-      if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x404u)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+    for (int i0 = 0; i0 < nkb && ok; i0 += kKbPer) {
 #pragma unroll
-      for (int c = 0; c < NT / 16; ++c) {
-        uint32_t r[16];
-        tmem_ld16(tmem_base + lane_base + buf * NT + 16 * c, r);
+      for (int h = 0; h < kHalves; ++h) {
+        uint32_t r[kKbPer][kCkB][16];
+#pragma unroll
+        for (int u = 0; u < kKbPer; ++u) {
+          const int i = i0 + u;
+          if (i < nkb && ok) {
+            const uint32_t buf = (uint32_t)(i % kBufs);
+            if (h == 0) {
+              if (!warp_wait(smem_u32(&tfull[buf]), (uint32_t)(i / kBufs) & 1, abort_flag,
+                             p.status, 0x404u))
+                ok = false;
+              else
+                tc_fence_after();
+            }
+            if (ok) {
+#pragma unroll
+              for (int c = 0; c < kCkB; ++c)
+                tmem_ld16(tmem_base + lane_base + buf * NT + 16 * (h * kCkB + c), r[u][c]);
+            }
+          }
+        }
         tmem_ld_wait();
+        if (ok) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = 16 * c + j;
-          acc[t] = fmaf(pval<DT>(r[j]), sa_s[i * NT + t] * swv, acc[t]);
+          for (int u = 0; u < kKbPer; ++u) {
+            const int i = i0 + u;
+            if (i < nkb) {
+              const float swv = sw_s[i];
+#pragma unroll
+              for (int c = 0; c < kCkB; ++c) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const int t = 16 * (h * kCkB + c) + j;
+                  acc[t] = fmaf(pval<DT>(r[u][c][j]), sa_s[i * NT + t] * swv, acc[t]);
+                }
+              }
+            }
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+      if (ok && lane == 0) {
+        for (int u = 0; u < kKbPer && i0 + u < nkb; ++u)
+          mbar_arrive(smem_u32(&tempty[(i0 + u) % kBufs]));
+      }
     }
-    (void)ok;
-    named_bar(1, 128);                 // all four epilogue warps decide together
+    // this warp has read TMEM for the last time: the MMA warp may free it
+    tc_fence_before();
+    named_bar_arrive(2, 160);
     if (p.cluster) {
-      // partial of this split -> own shared memory, [token][row]; the stage
-      // ring is free: every MMA has completed and consumed its loads
-      float* part_s = reinterpret_cast<float*>(smem);
-      const int row = 32 * q + lane;
+      // push this thread's row partial to the CTA that reduces the row:
+      // slot [source rank][token][row within the owner's share] of the
+      // owner's slot array, then one arrival on the owner's mbarrier
+      cluster_wait();                             // start-up barrier: peers are set up
+      const int rows_per = BN_W / p.splits;
+      const int r = 32 * q + lane;
+      const int owner = r / rows_per, rr = r - owner * rows_per;
+      const uint32_t my = cluster_rank();
+      if (!*abort_flag) {
+        constexpr int kNtp = L::kNtp;
+        const uint32_t dst = mapa_shared(smem_u32(slots), (uint32_t)owner) +
+                             4u * (uint32_t)(((int)my * rows_per + rr) * kNtp);
 #pragma unroll
-      for (int t = 0; t < NT; ++t) part_s[t * BN_W + row] = acc[t];
-    } else if (!*abort_flag) {
+        for (int c = 0; c < NT / 4; ++c)
+          if (4 * c < p.M)
+            st_dsmem_v4(dst + 16u * (uint32_t)c, acc[4 * c], acc[4 * c + 1], acc[4 * c + 2],
+                        acc[4 * c + 3]);
+      }
+      mbar_arrive_cluster(mapa_shared(smem_u32(&red[0]), (uint32_t)owner));
+      // this CTA's rows: all S sources x rows_per rows have arrived
+      const bool got = mbar_wait_cluster(smem_u32(&red[0]), 0, abort_flag, p.status, 0x405u);
+      if (got && !*abort_flag) {
+        // thread -> (row r2 of this CTA's share, token quads tq, tq + ng, ...)
+        constexpr int kNtp = L::kNtp;
+        const int r2 = et % rows_per, ng = 128 / rows_per;
+        const int64_t nn = (int64_t)tile * BN_W + (int)my * rows_per + r2;
+        const float b = (p.bias && nn < p.N) ? bf16_bits_to_float(p.bias[nn]) : 0.f;
+        const int quads = (int)((p.M + 3) / 4);
+        for (int tq = et / rows_per; tq < quads; tq += ng) {
+          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int src = 0; src < p.splits; ++src) {
+            const float4 v =
+                *reinterpret_cast<const float4*>(slots + (src * rows_per + r2) * kNtp + 4 * tq);
+            sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+          }
+          if (nn < p.N) {
+            const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (4 * tq + j < p.M)
+                p.out[(int64_t)(4 * tq + j) * p.ldo + nn] = float_to_bf16_bits(vals[j] + b);
+          }
+        }
+      }
+    } else {
+      // the four epilogue warps take one decision on abort (a consistent
+      // snapshot, as the named barriers below need all of them)
+      named_bar(1, 128);
+      if (et == 0) *epi_abort = *abort_flag;
+      named_bar(1, 128);
+      if (*epi_abort) return;
       const bool n_ok = n < p.N;
       if (p.splits == 1) {
         if (n_ok) {
@@ -335,48 +466,10 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
       }
     }
+    return;
   }
-
-  if (p.cluster) {
-    // every thread of every CTA in the cluster arrives: the partials are
-    // published, then each CTA reduces its share of rows in split order
-    cluster_sync_all();
-    const int S = p.splits;
-    const int rows_per = BN_W / S;             // 16, 32 or 64
-    const int quads = rows_per / 4;
-    const int c = (int)cluster_rank();
-    const float* part_s = reinterpret_cast<const float*>(smem);
-    const int items = (int)p.M * quads;
-    if (!*abort_flag) {
-      for (int it = threadIdx.x; it < items; it += kThreads) {
-        const int t = it / quads, qd = it - t * quads;
-        const int r0 = c * rows_per + 4 * qd;
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < S; ++src) {
-          const float4 v = ld_dsmem_f4(part_s + t * BN_W + r0, (uint32_t)src);
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        }
-        const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int64_t nn = (int64_t)tile * BN_W + r0 + j;
-          if (nn < p.N) {
-            const float b = p.bias ? bf16_bits_to_float(p.bias[nn]) : 0.f;
-            p.out[(int64_t)t * p.ldo + nn] = float_to_bf16_bits(vals[j] + b);
-          }
-        }
-      }
-    }
-    // keep this CTA's shared memory alive until every peer has read it
-    cluster_sync_all();
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, tmem_cols<NT>());
-  }
+  // producer and MMA warps: complete their part of the start-up barrier
+  if (p.cluster) cluster_wait();
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -386,15 +479,14 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 EncodeTiledFn enc() {
   static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
             cudaSuccess && q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
+  });
   return fn;
 }
 
@@ -409,13 +501,6 @@ bool tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
-}
-
-int num_sms() {
-  int dev = 0, v = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-  return v > 0 ? v : 148;
 }
 
 // Largest number of clusters of `S` CTAs of this kernel the device can hold
@@ -441,7 +526,8 @@ int max_active_clusters(int S) {
     cfg.attrs = &at;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_decode_kernel<DT, NT>, &cfg) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_decode_kernel<DT, NT>, &cfg) !=
+            cudaSuccess ||
         n < 1) {
       cudaGetLastError();
       n = 1;
@@ -452,13 +538,14 @@ int max_active_clusters(int S) {
 }
 
 // Split count for cluster mode: keep as many CTAs resident in the first wave
-// as possible (fewer waves first, then more resident CTAs, then larger S).
+// as possible (fewer waves first, then more resident CTAs, then larger S),
+// with at most max_kb K-blocks per split.  0 if no split count fits.
 template <int DT, int NT>
-int cluster_splits(int64_t tiles, int64_t Kb) {
-  int best = 2;
+int cluster_splits(int64_t tiles, int64_t Kb, int max_kb) {
+  int best = 0;
   double best_score = -1.0;
   for (int S = 8; S >= 2; S /= 2) {
-    if (S > Kb || (Kb + S - 1) / S > kMaxSplitKb) continue;
+    if (S > Kb || (Kb + S - 1) / S > max_kb) continue;
     const int64_t n = max_active_clusters<DT, NT>(S);
     const int64_t waves = (tiles + n - 1) / n;
     const double score = (double)std::min<int64_t>(n, tiles) * S / (double)waves;
@@ -479,14 +566,18 @@ cudaError_t launch_nt(const GemmArgs& a, const DecodePlan& plan_in, void* ws, bo
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kTotal);
   if (e != cudaSuccess) return e;
   DecodePlan plan = plan_in;
-  if (plan.cluster) plan.splits = cluster_splits<DT, NT>(plan.tiles, (a.K + BK - 1) / BK);
+  const int64_t Kb = (a.K + BK - 1) / BK;
+  if (plan.cluster) {
+    plan.splits = cluster_splits<DT, NT>(plan.tiles, Kb, kMaxSplitKb);
+    if (plan.splits == 0) return cudaErrorInvalidValue;
+  }
   CUtensorMap tW, tA;
   if (!tmap(&tW, a.qw, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.ldw, BN_W) ||
       !tmap(&tA, a.qa, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.lda, NT))
     return cudaErrorInvalidValue;
   DecParams p;
   p.sa = a.sa; p.sw = a.sw;
-  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK;
+  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = Kb;
   p.splits = plan.splits;
   p.cluster = plan.cluster ? 1 : 0;
   p.bias = static_cast<const uint16_t*>(a.bias);
@@ -533,7 +624,6 @@ cudaError_t launch_dt(const GemmArgs& a, const DecodePlan& plan, void* ws, bool 
 }
 
 }  // namespace
-
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K) {
   DecodePlan d;
   d.nt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
@@ -610,7 +700,6 @@ cudaError_t noalloc_scratch(void** ptr) {
 cudaError_t launch_gemm_decode(const GemmArgs& a, void* ws, bool pdl, cudaStream_t st) {
   if (a.M == 0 || a.N == 0) return cudaSuccess;
   const DecodePlan plan = decode_plan(a.M, a.N, a.K);
-  (void)num_sms;
   if (a.dtype == kInt8) return launch_dt<kInt8>(a, plan, ws, pdl, st);
   return launch_dt<kFp8>(a, plan, ws, pdl, st);
 }

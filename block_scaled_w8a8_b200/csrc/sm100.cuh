@@ -234,6 +234,23 @@ __device__ __forceinline__ void cluster_sync_all() {
                ::: "memory");
 }
 
+// The two halves of cluster_sync_all, for work placed between them.  Every
+// thread of every CTA must execute each exactly once per phase, in order.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Store four fp32 (16-byte aligned) to another CTA's shared memory.
+__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float a, float b, float c,
+                                            float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
+               "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // Address, in the cluster's shared window, of the variable at local shared
 // address `local` in the CTA of cluster rank `rank`.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t local, uint32_t rank) {

@@ -233,6 +233,68 @@ def test_linear_decode_path_with_dependent_launch(M):
     assert all(torch.equal(outs[0], o) for o in outs[1:])
 
 
+# Shapes on which bq_linear runs the fused decode kernel (the kernel quantises
+# its own K slice of x): M <= 32, at least 16 weight tiles, x 16-byte aligned
+# with a row stride that is a multiple of 8.  Partial K-blocks, K not a
+# multiple of 8 (row stride padded), ragged N and bias are all covered.
+FUSED_SHAPES = [(1, 2048, 4096, 4096), (5, 4096, 1000, 1000), (16, 2048, 1004, 1008),
+                (17, 3000, 4096, 4096), (32, 4096, 8192, 8192), (3, 2100, 300, 304)]
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,N,K,ldx", FUSED_SHAPES)
+def test_linear_fused_decode_vs_oracle(M, N, K, ldx, dtype):
+    xb = act_bits(M, K, 90 + M, 7, 25.0)
+    w = bq_synth.weights(N, K, 0.02, 91 + M).numpy()
+    qw, sw = oracle.quant_weight(w, 128, 128, dtype)
+    bias = oracle.bf16_from_f64(np.random.default_rng(M).normal(0, 0.5, N))
+    xpad = np.zeros((M, ldx), dtype=np.uint16)
+    xpad[:, :K] = xb
+    x = dev_bf16(xpad)[:, :K]
+    assert x.stride(0) == ldx
+    outs = [bq.linear(x, dev_u8(qw), dev_f32(sw), 128, 128, dtype, bias=dev_bf16(bias))
+            for _ in range(2)]
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    qa, sa = oracle.quant_act(xb, 128, dtype)
+    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bias)
+    assert_gemm_close(outs[0], ref, f"fused linear M={M} N={N} K={K}")
+    assert torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M", [1, 7, 32])
+def test_linear_fused_codes_exact_through_identity_weight(M, dtype):
+    """With W = identity (code of 1.0, block scale 1) each output is
+    bf16(fl32(q[t, n] * sa[t, n // 128])): one product, rounded to fp32 by the
+    kernel's promotion FMA, then to bf16.  Neighbouring INT8 codes (and e4m3
+    codes) differ by at least 1/127 (1/8) relatively, more than a bf16 ulp,
+    so any wrong code or misplaced swizzle slot of the fused quantiser shows
+    as an exact mismatch against the oracle's codes."""
+    N = K = 2048
+    xb = act_bits(M, K, 300 + M, 11, 40.0)
+    one = 1 if dtype == INT8 else int(oracle.e4m3_encode(np.array([1.0]))[0])
+    qw = np.zeros((N, K), dtype=np.uint8)
+    qw[np.arange(N), np.arange(K)] = one
+    sw = np.ones((N // 128, K // 128), dtype=np.float32)
+    out = bq.linear(dev_bf16(xb), dev_u8(qw), dev_f32(sw), 128, 128, dtype)
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    qa, sa = oracle.quant_act(xb, 128, dtype)
+    vals = oracle.code_values(qa, dtype).astype(np.float32)
+    expect = vals * np.repeat(sa, 128, axis=1).astype(np.float32)      # fp32 product
+    expect_bits = oracle.bf16_from_f64(expect.astype(np.float64))
+    got = host_bits(out)
+    # compared as values: the split sum starts from +0, so a -0 product (the
+    # e4m3 code 0x80) comes out as +0, as in the oracle's sum
+    bad = np.argwhere(oracle.bf16_to_f64(got) != oracle.bf16_to_f64(expect_bits))
+    detail = [(int(t), int(n), hex(int(qa[t, n])), float(vals[t, n]),
+               float(oracle.bf16_to_f64(got[t, n])), float(oracle.bf16_to_f64(expect_bits[t, n])))
+              for t, n in bad[:8]]
+    assert len(bad) == 0, \
+        f"{len(bad)} outputs differ from bf16(code * scale): (t, n, code, value, got, want) {detail}"
+
+
 def test_linear_decode_in_cuda_graph():
     M, N, K = 32, 1024, 2048
     xb = act_bits(M, K, 77, 20, 30.0)

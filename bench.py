@@ -40,6 +40,25 @@ METRIC = "block-scaled W8A8 GEMM TOPS & weight GB/s; % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def load_traffic(kernel_source: str):
+    """DRAM bytes per launch of the roofline kernel from the committed ncu
+    record (profiles/roofline_traffic.json), or (None, why) when there is no
+    record or the kernel source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "block_scaled_w8a8_b200", "csrc", rec["source_file"])
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None, "no ncu record"
+    if rec["source_file"] != kernel_source or rec["source_sha256"] != digest:
+        return None, "kernel changed since the ncu capture"
+    return float(rec["dram_bytes_per_launch"]), rec["capture"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -54,21 +73,32 @@ def load_peaks():
 # --------------------------------------------------------------------------
 
 class Dist:
-    def __init__(self, n_gpus: int):
+    """One process per GPU (torchrun env). Replicas only: ranks run the same
+    workload on their own GPU with no data-path collective; the barrier and
+    the max over ranks are the timing plumbing. NCCL on GPUs, gloo on CPU."""
+
+    def __init__(self, n_gpus: int, backend: str | None = None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.n_gpus = n_gpus
         self.pg = None
+        self.device = torch.device("cpu")
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                self.device = torch.device("cuda", self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                        device_id=self.device)
+            else:
+                dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
             self.pg = dist
         elif torch.cuda.is_available():
             torch.cuda.set_device(0)
+            self.device = torch.device("cuda", 0)
 
     def barrier(self):
         if self.pg:
@@ -77,13 +107,19 @@ class Dist:
     def max(self, v: float) -> float:
         if not self.pg:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def whole_job_rate(world: int, steps: int, units_per_step: float, seconds: float) -> float:
+    """Units all ranks processed per second: every rank runs `steps` steps of
+    `units_per_step`, and `seconds` is the slowest rank's time (weak scaling)."""
+    return world * steps * units_per_step / seconds
 
 
 # --------------------------------------------------------------------------
@@ -264,18 +300,20 @@ def bench_decode(args, dist, bq, peaks, stream):
     t_e2e = timed_graph_steps(e2e_graphs, args.steps, args.warmup, stream, dist)
 
     n = dist.world
-    value = n * args.steps * step_bytes / t / 1e9
+    traffic, traffic_src = load_traffic("gemm_decode.cu")
+    value = whole_job_rate(n, args.steps, step_bytes, t) / 1e9
     gemm_launch_s = t_gemm / (args.steps * len(Ms))
     achieved = gemm_bytes / len(Ms) / gemm_launch_s / 1e9
     res = {
         "value": value, "unit": "GB/s", "ms_per_step": 1e3 * t / args.steps,
         "roofline": {"bound": "hbm", "kernel": "block-scaled GEMM (decode shapes)",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "traffic_source": traffic_src,
                      "algorithmic_bytes_per_launch": gemm_bytes / len(Ms),
                      "avg_launch_us": 1e6 * gemm_launch_s},
         "quant_us_per_launch": 1e6 * t_quant / (args.steps * len(Ms)),
-        "e2e": {"value": n * args.steps * step_bytes / t_e2e / 1e9, "unit": "GB/s",
+        "e2e": {"value": whole_job_rate(n, args.steps, step_bytes, t_e2e) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": sum(2 * M * K for M in Ms),
                 "d2h_bytes_per_step": sum(2 * M * N for M in Ms)},
         "gpu_launches": args.steps * 2 * len(Ms),
@@ -326,7 +364,7 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
     peak = 2.0 * peaks["bf16_tflops"]
     ach = ops / (t_gemm / args.steps) / 1e12
     del graphs, gemm_graphs
-    return {"value": dist.world * args.steps * ops / t / 1e12, "unit": "TOPS",
+    return {"value": whole_job_rate(dist.world, args.steps, ops, t) / 1e12, "unit": "TOPS",
             "ms_per_step": 1e3 * t / args.steps,
             "roofline": {"bound": "tensor", "kernel": "tcgen05 block-scaled GEMM",
                          "achieved": ach, "peak": peak, "unit": "TFLOP/s" if cfg.dtype else
@@ -434,7 +472,7 @@ def bench_moe(args, dist, bq, peaks, stream):
     peak = 2.0 * peaks["bf16_tflops"]
     ach = ops / (t_g / steps) / 1e12
     del g, gg
-    return {"value": dist.world * steps * ops / t / 1e12, "unit": "TOPS",
+    return {"value": whole_job_rate(dist.world, steps, ops, t) / 1e12, "unit": "TOPS",
             "ms_per_step": 1e3 * t / steps, "steps": steps,
             "roofline": {"bound": "tensor", "kernel": "tcgen05 grouped GEMM (w13 + w2)",
                          "achieved": ach, "peak": peak, "unit": "TOPS", "frac": ach / peak,

@@ -186,6 +186,12 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   const int nkb = kb1 - kb0;
   const int first = min(nkb, kStages);
 
+  // this split's weight scales: constant data, requested before the weight
+  // tiles so that they do not queue behind them in the memory system; the
+  // epilogue warps store them to shared memory before their first use
+  const int swi = (int)threadIdx.x - 64;
+  const float sw_reg =
+      (swi >= 0 && swi < nkb) ? __ldg(p.sw + (int64_t)tile * p.Kb + kb0 + swi) : 0.f;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
@@ -199,6 +205,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     mbar_init(smem_u32(&red[0]), BN_W);     // one arrival per pushed row
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  __syncthreads();                    // barriers initialised, scale loads issued
+  if (threadIdx.x == 0) {
     // The weights do not depend on the preceding kernel: the first stages are
     // requested before this CTA waits for its activations.
     tma_prefetch_desc(&tmW);
@@ -209,9 +218,6 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
     tma_prefetch_desc(&tmA);
   }
-  // this split's weight scales: constant data, read before the wait
-  if (threadIdx.x >= 64 && threadIdx.x - 64 < nkb)
-    sw_s[threadIdx.x - 64] = __ldg(p.sw + (int64_t)tile * p.Kb + kb0 + (threadIdx.x - 64));
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), tmem_cols<NT>());
   // start-up cluster barrier: the peers' mbarriers are initialised before
   // anyone arrives on them remotely (waited on just before the push)
@@ -310,6 +316,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     const int et = threadIdx.x - 64;              // 0..127
     const int64_t n = (int64_t)tile * BN_W + 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    if (et < nkb) sw_s[et] = sw_reg;
     grid_dep_wait();                              // sa is written by the quantiser
     for (int idx = et; idx < nkb * NT; idx += 128) {
       const int kbl = idx / NT, t = idx % NT;

@@ -5,13 +5,17 @@
 // quantization doc, "GEMM backends for FP4/FP8"), for block_n = block_k = 128.
 //
 // Design (persistent, warp-specialised, one CTA per SM):
-//   warp 0      TMA producer: per K-block, one 128x128 A tile and one BNx128
-//               W tile (K-major, 128-byte swizzle) into an S-stage ring.
+//   warps 0, 2  TMA producers: per K-block, warp 0 loads one 128x128 A tile
+//               and warp 2 one BNx128 W tile (K-major, 128-byte swizzle) into
+//               an S-stage ring (one issuing thread alone cannot sustain the
+//               L2->SMEM rate a K-block needs).
 //   warp 1      MMA issuer (lane 0): 4 x tcgen05.mma (K = 32 each) per K-block
 //               into a TMEM buffer; the buffer holds exactly one K-block's
 //               partial P_kb (int32 for kind::i8, fp32 for kind::f8f6f4).
-//               Two TMEM buffers alternate so the MMA of block kb+1 overlaps
-//               the promotion of block kb.  Also owns the TMEM allocation.
+//               Four TMEM buffers (all 512 columns) rotate, so the MMA runs
+//               up to three K-blocks ahead of the promotion and the TMEM
+//               hand-off latency stays off the critical path.  Also owns the
+//               TMEM allocation.
 //   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
 //               per thread) and columns [32*h, 32*h+32), h = (w-4)/4; it
 //               promotes acc += P_kb * (sa[kb][m] * sw[nb][kb]) in fp32
@@ -59,14 +63,15 @@ using tc::wrow_block;
 using tc::make_tmap;
 using tc::sm_count;
 using tc::encode_fn;
-constexpr int kThreads = 640;        // 20 warps: producer, MMA, 2 idle, 16 epilogue
+constexpr int kThreads = 640;        // 20 warps: A producer, MMA, W producer, idle, 16 epilogue
 constexpr int kEpiWarps = 16;
+constexpr int kTBufs = 4;            // TMEM accumulators of BN columns (4 x 128 = all 512)
 
 template <int BN, int S>
 struct Smem {
   static constexpr uint32_t kA = BM * BK, kB = BN * BK;
   static constexpr uint32_t kStages = S * (kA + kB);
-  static constexpr uint32_t kBars = (2 * S + 4 + 2) * 8;
+  static constexpr uint32_t kBars = (2 * S + 2 * kTBufs + 2) * 8;
   static constexpr uint32_t kMisc = 8 + 2 * (kMaxE + 1) * 4;
   static constexpr uint32_t kTotal = 1024 + kStages + kBars + kMisc;
 };
@@ -85,9 +90,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + 2;
-  uint64_t* drain = bars + 2 * S + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 6);
+  uint64_t* tempty = bars + 2 * S + kTBufs;
+  uint64_t* drain = bars + 2 * S + 2 * kTBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kTBufs + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* off_s = reinterpret_cast<int*>(tmem_slot + 2);
   int* tp_s = off_s + (kMaxE + 1);
@@ -97,10 +102,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&full[s]), 2);            // the A producer and the B producer
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kTBufs; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
       mbar_init(smem_u32(&tempty[b]), kEpiWarps);
     }
@@ -108,21 +113,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmB);
   // expert row ranges (sanitised: clamped to [0, M] and nondecreasing)
   if (threadIdx.x == 32) tc::load_expert_ranges<BM>(p, off_s, tp_s);
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 2 * BN);
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTBufs * BN);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tp_s[E];
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == 0 || warp == 2) {
+    // ---------------- TMA producers: warp 0 the A tiles, warp 2 the W tiles
+    // (one issuing thread sustains only part of the L2->SMEM rate a K-block
+    // needs; two issue in parallel) ----------------
+    const bool is_a = warp == 0;
     int stage = 0;
     uint32_t phase = 0;
     int issued_parity[S];
@@ -141,9 +147,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kA + L::kB);
-          tma_load_2d(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, smem_u32(&full[stage]));
-          tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, b_row, smem_u32(&full[stage]));
+          if (is_a) {
+            mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kA);
+            tma_load_2d(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, smem_u32(&full[stage]));
+          } else {
+            mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kB);
+            tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, b_row, smem_u32(&full[stage]));
+          }
         }
         issued_parity[stage] = (int)phase;
         if (++stage == S) {
@@ -171,7 +181,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     bool ok = true, issued_any = false;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       for (int kb = 0; kb < p.Kb; ++kb) {
-        const uint32_t buf = kcount & 1, tround = kcount >> 1;
+        const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
         if (!warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag, p.status, 0x302u) ||
             !warp_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x303u)) {
           ok = false;
@@ -232,7 +242,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
       float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
       for (int kb = 0; kb < p.Kb; ++kb) {
-        const uint32_t buf = kcount & 1, tround = kcount >> 1;
+        const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
         const float f = sa_next * sw_next;
         if (kb + 1 < p.Kb) {
           sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
@@ -303,7 +313,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    tmem_dealloc(tmem_base, kTBufs * BN);
   }
 }
 

@@ -251,19 +251,21 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tc_fence_after();
         const uint64_t f2 = pack2(f, f);
         const uint32_t taddr = tmem_base + lane_base + buf * TN + tcol;
+        // 16 columns per TMEM load: with kEpiCols accumulators live, larger
+        // chunks would not fit the register budget of 18 warps per SM
 #pragma unroll
-        for (int c = 0; c < kEpiCols / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(taddr + 32 * c, r);
+        for (int c = 0; c < kEpiCols / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(taddr + 16 * c, r);
           tmem_ld_wait();
-          if (c == kEpiCols / 32 - 1) {
+          if (c == kEpiCols / 16 - 1) {
             // every column of this warp is in registers: hand the buffer back
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + 8u * buf);
           }
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             uint64_t x;
             if constexpr (DT == kInt8) {
               x = ((uint64_t)(r[2 * i + 1] + kMagicBits) << 32) |
@@ -272,7 +274,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             } else {
               x = ((uint64_t)r[2 * i + 1] << 32) | (uint64_t)r[2 * i];
             }
-            acc[16 * c + i] = fma2(x, f2, acc[16 * c + i]);
+            acc[8 * c + i] = fma2(x, f2, acc[8 * c + i]);
           }
         }
         ++kcount;

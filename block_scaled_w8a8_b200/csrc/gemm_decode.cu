@@ -13,7 +13,9 @@
 //    weight tile through a TMA ring, small enough that two CTAs share an SM;
 //  * before griddepcontrol.wait (programmatic dependent launch) a CTA issues
 //    its first weight stages and reads its weight scales: neither depends on
-//    the preceding kernel, so both overlap that kernel's tail.  The next
+//    the preceding kernel, so both overlap that kernel's tail.  The weights
+//    are read exactly once and loaded with an L2 evict-first policy, so they
+//    do not push the small, reused tensors of neighbouring layers out of L2.  The next
 //    kernel is released once this CTA's first activation tile has arrived,
 //    so its weight stream does not queue ahead of this CTA's activation reads;
 //  * per-K-block promotion in the epilogue warps (one weight row per thread,
@@ -213,8 +215,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     tma_prefetch_desc(&tmW);
     for (int i = 0; i < first; ++i) {
       mbar_arrive_expect_tx(smem_u32(&full[i]), L::kStage);
-      tma_load_2d(smem_u32(smem + i * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
-                  smem_u32(&full[i]));
+      tma_load_2d_hint(smem_u32(smem + i * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
+                       smem_u32(&full[i]), policy_evict_first());
     }
     tma_prefetch_desc(&tmA);
   }
@@ -248,8 +250,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kStage);
-        tma_load_2d(smem_u32(smem + stage * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
-                    smem_u32(&full[stage]));
+        tma_load_2d_hint(smem_u32(smem + stage * L::kStage), &tmW, (kb0 + i) * BK, tile * BN_W,
+                         smem_u32(&full[stage]), policy_evict_first());
         tma_load_2d(smem_u32(smem + stage * L::kStage + L::kW), &tmA, (kb0 + i) * BK, 0,
                     smem_u32(&full[stage]));
       }

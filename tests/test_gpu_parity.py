@@ -45,6 +45,11 @@ def act_bits(M, K, seed, n_out=0, scale=1.0):
     (3, 700, 256, 0),       # group longer than 128 (two-pass)
     (7, 333, 100, 3),       # group not a multiple of 4 (scalar path)
     (1, 1, 128, 0),
+    # many rows: the half-warp-per-group path (16-byte loads, K % 8 == 0)
+    (300, 1000, 128, 8),    # partial last group (104 elements), padded stride
+    (129, 4096, 128, 0),    # odd row count: a half-empty last pair of groups
+    (256, 136, 128, 0),     # second group of 8 elements
+    (130, 1004, 128, 4),    # K % 8 != 0: the one-warp-per-group path
 ])
 def test_quant_act_bit_exact(dtype, M, K, gk, pad):
     xb = act_bits(M, K + pad, 11 + M, max(1, (K + pad) // 100), 30.0)

@@ -19,13 +19,14 @@
 //   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
 //               per thread) and columns [BN/4*h, BN/4*(h+1)), h = (w-4)/4; it
 //               promotes acc += P_kb * (sa[kb][m] * sw[nb][kb]) in fp32
-//               registers with packed f32x2 arithmetic, frees the buffer, and
+//               registers (scalar FADD/FFMA: measured faster here than the
+//               packed f32x2 forms), frees the buffer, and
 //               after the last K-block adds the bias and stores bf16.
 // INT8 promotion without the int->float conversion unit: since
 // |P_kb| <= 128 * 128 * 128 < 2^22, the integer sum P_kb + 0x4B400000 (an
 // integer add on the ALU pipe) has the bits of the float 12582912 + P_kb
 // exactly, so one FADD recovers P_kb exactly and one FFMA promotes it (FMA
-// pipe, packed two per instruction).
+// pipe).
 // A tile scheduler walks (expert, m-block, n-block) tiles; a dense problem is
 // one expert.  The grouped (MoE) problem reads its expert row ranges from
 // device memory, so no host read-back is needed.  Rows of a tile past the
@@ -229,7 +230,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint32_t kcount = 0;
     int e_hint = 0;
     bool ok = true;
-    const uint64_t neg_magic2 = pack2(-kMagic, -kMagic);
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       int e, mb, nb;
       decode_tile<BM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
@@ -239,9 +239,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int64_t n0 = (int64_t)nb * BN + CW * half;
       const float* sw_e = p.sw + (int64_t)e * p.sw_expert_stride;
       const int64_t swrow = n0 < p.N ? wrow_block(n0, p.seam, p.N) * p.Kb : 0;
-      uint64_t acc[CW / 2];
+      float accf[CW];
 #pragma unroll
-      for (int i = 0; i < CW / 2; ++i) acc[i] = 0ull;
+      for (int i = 0; i < CW; ++i) accf[i] = 0.f;
       float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
       float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
       for (int kb = 0; kb < p.Kb; ++kb) {
@@ -257,7 +257,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_base + buf * BN + tcol;
-        const uint64_t f2 = pack2(f, f);
         // CW columns in chunks of RC: all at once for 32, 16 at a time for 64
         // (with 64 accumulators live, larger chunks do not fit the registers)
         constexpr int RC = CW <= 32 ? CW : 16;
@@ -274,14 +273,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
 #pragma unroll
           for (int i = 0; i < RC / 2; ++i) {
-            uint64_t x;
+            float x0, x1;
             if constexpr (DT == kInt8) {
-              x = ((uint64_t)(r[2 * i + 1] + kMagicBits) << 32) | (uint64_t)(r[2 * i] + kMagicBits);
-              x = add2(x, neg_magic2);                           // exact P_kb
+              x0 = __uint_as_float(r[2 * i] + kMagicBits) - kMagic;
+              x1 = __uint_as_float(r[2 * i + 1] + kMagicBits) - kMagic;
             } else {
-              x = ((uint64_t)r[2 * i + 1] << 32) | (uint64_t)r[2 * i];
+              x0 = __uint_as_float(r[2 * i]);
+              x1 = __uint_as_float(r[2 * i + 1]);
             }
-            acc[(RC / 2) * c + i] = fma2(x, f2, acc[(RC / 2) * c + i]);
+            accf[RC * c + 2 * i] = fmaf(x0, f, accf[RC * c + 2 * i]);
+            accf[RC * c + 2 * i + 1] = fmaf(x1, f, accf[RC * c + 2 * i + 1]);
           }
         }
         ++kcount;
@@ -297,8 +298,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t w[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              float v0 = __uint_as_float((uint32_t)acc[j / 2 + h]);
-              float v1 = __uint_as_float((uint32_t)(acc[j / 2 + h] >> 32));
+              float v0 = accf[j + 2 * h];
+              float v1 = accf[j + 2 * h + 1];
               if (p.bias) {
                 v0 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h));
                 v1 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h + 1));
@@ -311,7 +312,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int j = 0; j < CW; ++j) {
             if (n0 + j < p.N) {
-              float x = __uint_as_float((uint32_t)(acc[j / 2] >> (32 * (j & 1))));
+              float x = accf[j];
               if (p.bias) x += bf16_bits_to_float(__ldg(p.bias + n0 + j));
               orow[j] = float_to_bf16_bits(x);
             }

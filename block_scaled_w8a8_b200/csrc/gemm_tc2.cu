@@ -13,11 +13,11 @@
 // CTAs' operands, so the L2 traffic per output drops to 3/4 (TN = 128) or
 // 1/2 (TN = 256) of the single-CTA kernel's.
 //
-// Roles (persistent; one pair per two SMs; 18 warps per CTA):
-//   warp 0      TMA producer of each CTA: its A rows [128r, 128r+128) and W
-//               rows [TN/2 r, TN/2 (r+1)) of the pair tile, into an 8- or
-//               6-stage ring; completion is counted on the LEADER CTA's
-//               stage barrier (cta_group::2 loads, no multicast).
+// Roles (persistent; one pair per two SMs; 19 warps per CTA):
+//   warps 0, 18 TMA producers of each CTA: warp 0 its A rows [128r, 128r+128)
+//               and warp 18 its W rows [TN/2 r, TN/2 (r+1)) of the pair tile,
+//               into an 8- or 6-stage ring; completion is counted on the
+//               LEADER CTA's stage barrier (cta_group::2 loads, no multicast).
 //   warp 1      leader: issues the pair MMAs (4 x K = 32 per K-block) into one
 //               of 512/TN TMEM buffers of TN columns and commits to the stage
 //               and TMEM barriers of both CTAs at once; both CTAs' warp 1 own
@@ -26,7 +26,8 @@
 //               its own CTA (one output row per thread) and TN/4 columns
 //               (w-2)/4; per K-block it promotes acc += P_kb * sa * sw in fp32
 //               (INT8: exact int->float by the 1.5 * 2^23 offset trick on the
-//               ALU and FMA pipes), releases the buffer to the leader, and
+//               ALU and FMA pipes; scalar FADD/FFMA), releases the buffer to
+//               the leader, and
 //               after the last K-block adds the bias and stores bf16.
 // The tile scheduler is the one of the single-CTA kernel with 256-row tiles:
 // dense problems are one expert, grouped (MoE) problems read their expert
@@ -59,7 +60,8 @@ using tc::kMagicBits;
 using tc::TcParams;
 
 constexpr int TM = 256;            // pair tile rows (128 per CTA)
-constexpr int kThreads = 576;      // 18 warps: producer, MMA, 16 epilogue
+constexpr int kThreads = 608;      // 19 warps: A producer, MMA, 16 epilogue, W producer
+constexpr int kWProducerWarp = 18;
 constexpr int kEpiWarps = 16;
 
 // Pair tile of 256 x TN: each CTA stages 128 rows of A and TN/2 rows of W
@@ -115,10 +117,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
+  if (warp == kWProducerWarp && lane == 0) tma_prefetch_desc(&tmB);
   if (threadIdx.x == 32) tc::load_expert_ranges<TM>(p, off_s, tp_s);
   if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), 512);
   // both CTAs' barriers exist before any load or commit can signal them
@@ -133,8 +133,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
   for (int s = 0; s < kStages; ++s) issued_parity[s] = -1;
 
-  if (warp == 0) {
-    // ---------------- TMA producer (both CTAs) ----------------
+  if (warp == 0 || warp == kWProducerWarp) {
+    // ---------------- TMA producers (both CTAs): warp 0 the A rows, warp 18
+    // the W rows (one issuing thread alone cannot sustain the L2 -> shared
+    // memory rate a K-block needs) ----------------
+    const bool is_a = warp == 0;
     const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
     int stage = 0;
     uint32_t phase = 0;
@@ -152,11 +155,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
         if (lane == 0) {
           // the leader expects the bytes of both CTAs on its stage barrier
-          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * L::kStage);
+          if (rank == 0 && is_a) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * L::kStage);
           const uint32_t bar = leader_full0 + 8u * (uint32_t)stage;
           uint8_t* st = sA + stage * L::kStage;
-          tma_load_2d_pair(smem_u32(st), &tmA, kb * BK, a_row, bar);
-          tma_load_2d_pair(smem_u32(st + L::kA), &tmB, kb * BK, b_row, bar);
+          if (is_a) tma_load_2d_pair(smem_u32(st), &tmA, kb * BK, a_row, bar);
+          else tma_load_2d_pair(smem_u32(st + L::kA), &tmB, kb * BK, b_row, bar);
         }
         issued_parity[stage] = (int)phase;
         if (++stage == kStages) {
@@ -165,7 +168,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
       }
     }
-    leader_drain = !ok;
+    if (is_a) leader_drain = !ok;
   } else if (warp == 1) {
     // ---------------- pair MMA issuer (leader only) ----------------
     if (rank == 0) {
@@ -219,7 +222,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const uint32_t tcol = (uint32_t)(kEpiCols * g);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
-    const uint64_t neg_magic2 = pack2(-kMagic, -kMagic);
     uint32_t kcount = 0;
     int e_hint = 0;
     bool ok = true;
@@ -232,9 +234,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const int64_t n0 = (int64_t)nb * TN + kEpiCols * g;
       const float* sw_e = p.sw + (int64_t)e * p.sw_expert_stride;
       const int64_t swrow = n0 < p.N ? tc::wrow_block(n0, p.seam, p.N) * p.Kb : 0;
-      uint64_t acc[kEpiCols / 2];
+      float accf[kEpiCols];
 #pragma unroll
-      for (int i = 0; i < kEpiCols / 2; ++i) acc[i] = 0ull;
+      for (int i = 0; i < kEpiCols; ++i) accf[i] = 0.f;
       float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
       float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
       for (int kb = 0; kb < p.Kb; ++kb) {
@@ -249,7 +251,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           break;
         }
         tc_fence_after();
-        const uint64_t f2 = pack2(f, f);
         const uint32_t taddr = tmem_base + lane_base + buf * TN + tcol;
         // 16 columns per TMEM load: with kEpiCols accumulators live, larger
         // chunks would not fit the register budget of 18 warps per SM
@@ -265,16 +266,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + 8u * buf);
           }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint64_t x;
-            if constexpr (DT == kInt8) {
-              x = ((uint64_t)(r[2 * i + 1] + kMagicBits) << 32) |
-                  (uint64_t)(r[2 * i] + kMagicBits);
-              x = add2(x, neg_magic2);               // exact P_kb
-            } else {
-              x = ((uint64_t)r[2 * i + 1] << 32) | (uint64_t)r[2 * i];
-            }
-            acc[8 * c + i] = fma2(x, f2, acc[8 * c + i]);
+          for (int i = 0; i < 16; ++i) {
+            float xv;
+            if constexpr (DT == kInt8) xv = __uint_as_float(r[i] + kMagicBits) - kMagic;  // exact
+            else xv = __uint_as_float(r[i]);
+            accf[16 * c + i] = fmaf(xv, f, accf[16 * c + i]);
           }
         }
         ++kcount;
@@ -289,8 +285,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             uint32_t w[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              float v0 = __uint_as_float((uint32_t)acc[j / 2 + h]);
-              float v1 = __uint_as_float((uint32_t)(acc[j / 2 + h] >> 32));
+              float v0 = accf[j + 2 * h];
+              float v1 = accf[j + 2 * h + 1];
               if (p.bias) {
                 v0 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h));
                 v1 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h + 1));
@@ -303,7 +299,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
           for (int j = 0; j < kEpiCols; ++j) {
             if (n0 + j < p.N) {
-              float x = __uint_as_float((uint32_t)(acc[j / 2] >> (32 * (j & 1))));
+              float x = accf[j];
               if (p.bias) x += bf16_bits_to_float(__ldg(p.bias + n0 + j));
               orow[j] = float_to_bf16_bits(x);
             }

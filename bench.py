@@ -223,8 +223,8 @@ def capture(fn, stream):
     return g
 
 
-def quant_weights(w, dtype, bq):
-    q, s = bq.quant_weight(w, 128, 128, dtype)
+def quant_weights(w, dtype, bq, bn=128, bk=128):
+    q, s = bq.quant_weight(w, bn, bk, dtype)
     return q, s
 
 
@@ -332,27 +332,28 @@ def bench_decode(args, dist, bq, peaks, stream):
 def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
     dev = torch.device("cuda", torch.cuda.current_device())
     M, N, K = cfg.M, cfg.N, cfg.K
+    bn, bk = cfg.block_n, cfg.block_k
     wq, wsc = [], []
     for i in range(n_rot):
         w = bq_synth.weights(N, K, cfg.w_std, cfg.seed + 10 * i, device=dev)
-        q, s = quant_weights(w, cfg.dtype, bq)
+        q, s = quant_weights(w, cfg.dtype, bq, bn, bk)
         wq.append(q)
         wsc.append(s)
         del w
     xs = [bq_synth.activations(M, K, cfg.seed + i, cfg.n_outliers, cfg.outlier_scale,
                                device=dev) for i in range(n_rot)]
     out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    Kb = cdiv(K, 128)
+    Kb = cdiv(K, bk)
     qa = torch.empty(M, K, dtype=torch.uint8, device=dev)
     sa = torch.empty(Kb, M, dtype=torch.float32, device=dev)
-    gws = bq.workspace(bq.gemm_workspace_size(M, N, K, 128, 128, cfg.dtype), dev)
+    gws = bq.workspace(bq.gemm_workspace_size(M, N, K, bn, bk, cfg.dtype), dev)
     torch.cuda.synchronize()
 
     def step(i, quant=True):
         def run():
             if quant:
-                bq.quant_act(xs[i], 128, cfg.dtype, q=qa, s=sa)
-            bq.gemm(qa, sa, wq[i], wsc[i], 128, 128, cfg.dtype, out=out, ws=gws)
+                bq.quant_act(xs[i], bk, cfg.dtype, q=qa, s=sa)
+            bq.gemm(qa, sa, wq[i], wsc[i], bn, bk, cfg.dtype, out=out, ws=gws)
         return run
 
     graphs = [capture(step(i), stream) for i in range(n_rot)]
@@ -372,7 +373,7 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
                          "peak_source": "2 x measured bf16 burst (8-bit dense = 2x bf16)",
                          "avg_launch_us": 1e6 * t_gemm / args.steps},
             "clocks": clk.summary(),
-            "config": {"workload": cfg.name, "M": M, "N": N, "K": K, "block": [128, 128],
+            "config": {"workload": cfg.name, "M": M, "N": N, "K": K, "block": [bn, bk],
                        "l2": f"{n_rot} rotating weight/activation copies"},
             "dtype": "fp8_e4m3" if cfg.dtype else "int8"}
 
@@ -561,7 +562,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bq", choices=["bq", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "fp8", "moe"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "fp8", "moe", "perchannel"])
     ap.add_argument("--no-sub", action="store_true", help="skip the sub-workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
     args = ap.parse_args()
@@ -583,10 +585,12 @@ def main():
             head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.PREFILL, 3)
         elif args.workload == "fp8":
             head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.FP8_LINEAR, 3)
+        elif args.workload == "perchannel":
+            head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.PER_CHANNEL, 3)
         else:
             head = bench_moe(args, dist, bq, peaks, stream)
         if not args.no_sub:
-            for name in ("prefill", "fp8", "moe"):
+            for name in ("prefill", "fp8", "moe", "perchannel"):
                 if name == args.workload:
                     continue
                 torch.cuda.empty_cache()
@@ -596,6 +600,9 @@ def main():
                 elif name == "fp8":
                     subs[name] = bench_linear_big(args, dist, bq, peaks, stream,
                                                   bq_synth.FP8_LINEAR, 3)
+                elif name == "perchannel":
+                    subs[name] = bench_linear_big(args, dist, bq, peaks, stream,
+                                                  bq_synth.PER_CHANNEL, 3)
                 else:
                     subs[name] = bench_moe(args, dist, bq, peaks, stream)
     bq.check_device_status()

@@ -79,7 +79,11 @@ struct Smem {
   static constexpr uint32_t kTotal = 1024 + kStages + kBars + kMisc;
 };
 
-template <int DT, int BN, int S>
+// ONEK: the scale grid has a single K-block (block_k >= K: per-token
+// activation scales, per-channel or per-row-block weight scales).  The MMAs
+// then accumulate a tile's whole K in TMEM and the epilogue promotes once per
+// tile, out = P * sa[m] * sw[n / block_n], instead of once per K-block.
+template <int DT, int BN, int S, bool ONEK>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcParams p) {
@@ -145,7 +149,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       decode_tile<BM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
       const int a_row = off_s[e] + mb * BM;
       const int b_row = e * (int)p.N + nb * BN;
-      for (int kb = 0; kb < p.Kb; ++kb) {
+      for (int kb = 0; kb < p.Kmma; ++kb) {
         if (!warp_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.status, 0x301u)) {
           ok = false;
           break;
@@ -184,9 +188,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int e_hint = 0;
     bool ok = true, issued_any = false;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      for (int kb = 0; kb < p.Kb; ++kb) {
+      for (int kb = 0; kb < p.Kmma; ++kb) {
+        // a TMEM buffer holds one K-block's partial, or (ONEK) a whole tile's
+        const bool unit_first = !ONEK || kb == 0;
+        const bool unit_last = !ONEK || kb == p.Kmma - 1;
         const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
-        if (!warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag, p.status, 0x302u) ||
+        if ((unit_first && !warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag,
+                                      p.status, 0x302u)) ||
             !warp_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x303u)) {
           ok = false;
           break;
@@ -198,13 +206,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * L::kB));
 #pragma unroll
           for (int j = 0; j < BK / 32; ++j)
-            mma<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc, j > 0 ? 1u : 0u);
+            mma<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc,
+                    (j > 0 || !unit_first) ? 1u : 0u);
           mma_commit(smem_u32(&empty[stage]));
-          mma_commit(smem_u32(&tfull[buf]));
+          if (unit_last) mma_commit(smem_u32(&tfull[buf]));
         }
         __syncwarp();
         issued_any = true;
-        ++kcount;
+        if (unit_last) ++kcount;
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
@@ -242,23 +251,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       float accf[CW];
 #pragma unroll
       for (int i = 0; i < CW; ++i) accf[i] = 0.f;
-      float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
-      float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
-      for (int kb = 0; kb < p.Kb; ++kb) {
+      if constexpr (ONEK) {
+        // the tile's whole K is in one TMEM buffer: one promotion per element,
+        // out = P * (sa[m] * sw[n / block_n]); the int32 sum over all of K is
+        // converted with one correctly rounded int -> float
         const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
-        const float f = sa_next * sw_next;
-        if (kb + 1 < p.Kb) {
-          sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
-          sw_next = n0 < p.N ? __ldg(sw_e + swrow + kb + 1) : 0.f;
-        }
-        if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x304u)) {
+        const float sa_m = row_ok ? p.sa[m] : 0.f;
+        if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x305u)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_base + buf * BN + tcol;
-        // CW columns in chunks of RC: all at once for 32, 16 at a time for 64
-        // (with 64 accumulators live, larger chunks do not fit the registers)
         constexpr int RC = CW <= 32 ? CW : 16;
 #pragma unroll
         for (int c = 0; c < CW / RC; ++c) {
@@ -272,20 +276,60 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
           }
 #pragma unroll
-          for (int i = 0; i < RC / 2; ++i) {
-            float x0, x1;
-            if constexpr (DT == kInt8) {
-              x0 = __uint_as_float(r[2 * i] + kMagicBits) - kMagic;
-              x1 = __uint_as_float(r[2 * i + 1] + kMagicBits) - kMagic;
-            } else {
-              x0 = __uint_as_float(r[2 * i]);
-              x1 = __uint_as_float(r[2 * i + 1]);
-            }
-            accf[RC * c + 2 * i] = fmaf(x0, f, accf[RC * c + 2 * i]);
-            accf[RC * c + 2 * i + 1] = fmaf(x1, f, accf[RC * c + 2 * i + 1]);
+          for (int i = 0; i < RC; ++i) {
+            const int64_t col = n0 + RC * c + i;
+            const float swc = col < p.N ? __ldg(sw_e + col / p.bn) : 0.f;
+            const float v = DT == kInt8 ? __int2float_rn((int)r[i]) : __uint_as_float(r[i]);
+            accf[RC * c + i] = v * (sa_m * swc);
           }
         }
         ++kcount;
+      } else {
+        float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
+        float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
+        for (int kb = 0; kb < p.Kb; ++kb) {
+          const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
+          const float f = sa_next * sw_next;
+          if (kb + 1 < p.Kb) {
+            sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
+            sw_next = n0 < p.N ? __ldg(sw_e + swrow + kb + 1) : 0.f;
+          }
+          if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x304u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + lane_base + buf * BN + tcol;
+          // CW columns in chunks of RC: all at once for 32, 16 at a time for 64
+          // (with 64 accumulators live, larger chunks do not fit the registers)
+          constexpr int RC = CW <= 32 ? CW : 16;
+#pragma unroll
+          for (int c = 0; c < CW / RC; ++c) {
+            uint32_t r[RC];
+            if constexpr (RC == 32) tmem_ld32(taddr, r);
+            else tmem_ld16(taddr + RC * c, r);
+            tmem_ld_wait();
+            if (c == CW / RC - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
+            }
+#pragma unroll
+            for (int i = 0; i < RC / 2; ++i) {
+              float x0, x1;
+              if constexpr (DT == kInt8) {
+                x0 = __uint_as_float(r[2 * i] + kMagicBits) - kMagic;
+                x1 = __uint_as_float(r[2 * i + 1] + kMagicBits) - kMagic;
+              } else {
+                x0 = __uint_as_float(r[2 * i]);
+                x1 = __uint_as_float(r[2 * i + 1]);
+              }
+              accf[RC * c + 2 * i] = fmaf(x0, f, accf[RC * c + 2 * i]);
+              accf[RC * c + 2 * i + 1] = fmaf(x1, f, accf[RC * c + 2 * i + 1]);
+            }
+          }
+          ++kcount;
+        }
       }
       if (!ok) break;
       if (row_ok && n0 < p.N) {
@@ -330,10 +374,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
-template <int DT, int BN, int S>
+template <int DT, int BN, int S, bool ONEK>
 cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   using L = Smem<BN, S>;
-  auto kern = gemm_tc_kernel<DT, BN, S>;
+  auto kern = gemm_tc_kernel<DT, BN, S, ONEK>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -350,7 +394,10 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   TcParams p;
   p.sa = a.sa; p.sa_rows = a.sa_rows;
   p.sw = a.sw; p.sw_expert_stride = a.sw_expert_stride;
-  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK; p.seam = a.seam;
+  p.M = a.M; p.N = a.N; p.K = a.K; p.seam = a.seam;
+  p.Kmma = (a.K + BK - 1) / BK;
+  p.Kb = ONEK ? 1 : p.Kmma;              // K-blocks of the scale grid
+  p.bn = a.bn;
   p.offsets = a.offsets; p.E = (int)a.E;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;
@@ -370,7 +417,11 @@ bool tc_supported(const GemmArgs& a, char* why, size_t n) {
     if (why) snprintf(why, n, "tcgen05 path: %s", msg);
     return false;
   };
-  if (a.bn != 128 || a.bk != 128) return no("needs block_n = block_k = 128");
+  const bool onek = a.bk >= a.K;           // one scale block along K
+  if (!(a.bn == 128 && a.bk == 128) && !onek)
+    return no("needs block_n = block_k = 128, or block_k >= K (per-token scales)");
+  if (onek && a.seam != 0 && a.seam % a.bn != 0)
+    return no("with block_k >= K the gate/up seam must be a multiple of block_n");
   if (a.K < 1) return no("needs K >= 1");
   if (a.lda % 16 != 0 || a.ldw % 16 != 0) return no("row strides must be multiples of 16 bytes");
   if ((reinterpret_cast<uintptr_t>(a.qa) & 15) || (reinterpret_cast<uintptr_t>(a.qw) & 15))
@@ -388,12 +439,17 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   // a 128 x 128 tile (32 KB), and the L2 -> shared-memory feed is what bounds
   // this kernel on B200 (measured: FP8 +40%, INT8 +11% over 128 x 128).
   // Narrow problems keep 128-wide tiles.
+  // a single scale block along K (per-token / per-channel scales): promote
+  // once per tile instead of once per 128-wide K-block
+  const bool onek = a.bk >= a.K;
   if (a.N > 128) {
-    if (a.dtype == kInt8) return launch_typed<kInt8, 256, 4>(a, st);
-    return launch_typed<kFp8, 256, 4>(a, st);
+    if (a.dtype == kInt8)
+      return onek ? launch_typed<kInt8, 256, 4, true>(a, st) : launch_typed<kInt8, 256, 4, false>(a, st);
+    return onek ? launch_typed<kFp8, 256, 4, true>(a, st) : launch_typed<kFp8, 256, 4, false>(a, st);
   }
-  if (a.dtype == kInt8) return launch_typed<kInt8, 128, 6>(a, st);
-  return launch_typed<kFp8, 128, 6>(a, st);
+  if (a.dtype == kInt8)
+    return onek ? launch_typed<kInt8, 128, 6, true>(a, st) : launch_typed<kInt8, 128, 6, false>(a, st);
+  return onek ? launch_typed<kFp8, 128, 6, true>(a, st) : launch_typed<kFp8, 128, 6, false>(a, st);
 }
 
 }  // namespace bq

@@ -379,7 +379,7 @@ cudaError_t launch_pair_typed(const GemmArgs& a, cudaStream_t st) {
   TcParams p;
   p.sa = a.sa; p.sa_rows = a.sa_rows;
   p.sw = a.sw; p.sw_expert_stride = a.sw_expert_stride;
-  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK; p.seam = a.seam;
+  p.M = a.M; p.N = a.N; p.K = a.K; p.Kb = (a.K + BK - 1) / BK; p.Kmma = p.Kb; p.bn = 128; p.seam = a.seam;
   p.offsets = a.offsets; p.E = (int)a.E;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;

@@ -23,6 +23,8 @@ struct TcParams {
   const float* sa; int64_t sa_rows;             // activation scales [Kb][sa_rows]
   const float* sw; int64_t sw_expert_stride;    // weight scales [E][Nbs][Kb]
   int64_t M, N, K, Kb, seam;
+  int64_t Kmma;                                 // 128-wide K-blocks the MMAs walk
+  int64_t bn;                                   // weight-scale rows cover bn output columns
   const int32_t* offsets; int E;                // grouped: expert row ranges (device)
   const uint16_t* bias;
   uint16_t* out; int64_t ldo;

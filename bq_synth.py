@@ -18,6 +18,8 @@ blockwise FP8 linear layers, restated as synthetic inputs):
            A ~ N(0,1); seed 6
   moe      T = 4096, H = 4096, E = 8, top-2 from softmax of N(0,1) logits;
            w13 [8, 28672, 4096], w2 [8, 4096, 14336] ~ N(0, 0.015); seed 7
+  perchannel  the prefill shape with block_n = 1, block_k = K (per-token and
+           per-channel scales); seed 8
 
 Generators use torch.Generator so that the same recipe runs on the CPU (for
 oracle comparisons) or directly on a CUDA device (for large benchmarks).
@@ -76,6 +78,10 @@ PREFILL = Linear("prefill_int8_m4096_n14336_k4096", 4096, 14336, 4096, 0.015,
                  one_percent(4096), 30.0, INT8, 5)
 FP8_LINEAR = Linear("fp8_e4m3_m2048_n4096_k14336", 2048, 4096, 14336, 0.01, 0, 1.0, FP8, 6)
 MOE = MoE("moe_int8_t4096_h4096_i14336_e8_top2", 4096, 4096, 14336, 8, 2, 0.015, 7)
+# the degenerate case of the block layout: one scale per token (block_k = K)
+# and one per output channel (block_n = 1), on the prefill shape
+PER_CHANNEL = Linear("perchannel_int8_m4096_n14336_k4096", 4096, 14336, 4096, 0.015,
+                     one_percent(4096), 30.0, INT8, 8, block_n=1, block_k=4096)
 
 
 def _gen(seed: int, device) -> torch.Generator:

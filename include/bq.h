@@ -84,7 +84,7 @@ typedef enum bq_path {
     BQ_PATH_SIMT = 1,     /* generic CUDA-core kernel: any shape/stride */
     BQ_PATH_TCGEN05 = 2,  /* TMA + tcgen05 tensor-core kernel (large M) */
     BQ_PATH_DECODE = 3,   /* split-K weight-streaming kernel (small M) */
-    BQ_PATH_TCGEN05_1CTA = 4,  /* force the 1-CTA 128x128-tile tcgen05 kernel */
+    BQ_PATH_TCGEN05_1CTA = 4,  /* force the 1-CTA tcgen05 kernel (128x256 tiles) */
     BQ_PATH_TCGEN05_2CTA = 5,  /* force the CTA-pair 256x256-tile kernel */
     BQ_PATH_GEMV = 6      /* CUDA-core weight-streaming kernel, INT8, M <= 8
                              (forced only) */
@@ -178,6 +178,15 @@ bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_
  * qw: codes [N, K] (row stride ldw >= K), sw: fp32 [ceil(N/block_n)][Kb];
  * bias: bf16 [N] or NULL; out: bf16 [M, N] (row stride ldo >= N).
  * block_k <= 65536 keeps INT8 block partials exact in int32.
+ * Kernels (BQ_PATH_AUTO): block_n = block_k = 128 with M <= 128 runs the
+ *   split-K decode kernel; M > 128 runs the tcgen05 kernel, which promotes
+ *   each 128-wide K-block.  block_k >= K (one scale per token and per
+ *   block_n rows of W: per-token / per-channel W8A8 with block_n = 1) also
+ *   runs the tcgen05 kernel for M > 128, which then accumulates all of K in
+ *   tensor memory and promotes once (the int32 sum is rounded once to fp32).
+ *   The tensor-core kernels need 16-byte aligned operands with row strides
+ *   that are multiples of 16 bytes; everything else runs the CUDA-core
+ *   kernel.
  * workspace: device memory of at least bq_gemm_workspace_size bytes (may be
  *   NULL when that size is 0).  Its first 64 KiB hold arrival counters: they
  *   must be zero before the workspace is first used, and every completed

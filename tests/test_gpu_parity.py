@@ -18,6 +18,7 @@ from gpu_util import (assert_codes_equal, assert_combine_close, assert_gemm_clos
 pytestmark = pytest.mark.gpu
 
 INT8, FP8 = bq.INT8, bq.FP8_E4M3
+cdiv = bq_synth.cdiv
 
 
 @pytest.fixture(autouse=True)
@@ -500,3 +501,50 @@ def test_bad_expert_id_is_reported():
         bq.check_device_status()
     assert ei.value.status == bq.ERR_INVALID_ARG
     assert off.cpu().numpy()[-1] == 4      # the two bad pairs are placed nowhere
+
+
+# --------------------------------------------------------------------------
+# one scale block along K: per-token activations, per-channel (block_n = 1)
+# or per-row-block weights -- the W8A8 degenerate case of the block layout
+# --------------------------------------------------------------------------
+
+ONEK_SHAPES = [(300, 512, 512, 1), (1024, 1000, 1000, 1), (260, 768, 4096, 128),
+               (513, 2048, 1024, 1)]
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,N,K,bn", ONEK_SHAPES)
+@pytest.mark.parametrize("path", [bq.PATH_AUTO, bq.PATH_TCGEN05_1CTA])
+def test_one_scale_block_along_k(path, M, N, K, bn, dtype):
+    xb = act_bits(M, K, 500 + M, max(1, K // 100), 30.0)
+    w = bq_synth.weights(N, K, 0.02, 501 + N).numpy()
+    bias = oracle.bf16_from_f64(np.random.default_rng(N).normal(0, 0.5, N))
+    qa, sa = oracle.quant_act(xb, K, dtype)                 # one scale per token
+    qw, sw = oracle.quant_weight(w, bn, K, dtype)           # one scale per bn rows
+    assert sa.shape == (M, 1) and sw.shape == (cdiv(N, bn), 1)
+    # the GPU's quantisers give the same codes and scales
+    qg, sg = bq.quant_act(dev_bf16(xb), K, dtype)
+    qwg, swg = bq.quant_weight(torch.from_numpy(w).cuda(), bn, K, dtype)
+    torch.cuda.synchronize()
+    assert_codes_equal(qg, qa, "per-token codes")
+    assert_scales_equal(sg, sa, "per-token scales")
+    assert_codes_equal(qwg, qw, "weight codes")
+    assert np.array_equal(swg.cpu().numpy().view(np.uint32), sw.view(np.uint32))
+    bq.set_path(path)
+    try:
+        if path == bq.PATH_TCGEN05_1CTA and K % 16 != 0:
+            # TMA rows must be multiples of 16 bytes: the forced path refuses
+            with pytest.raises(bq.BqError) as ei:
+                bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), bn, K, dtype)
+            assert ei.value.status == bq.ERR_UNSUPPORTED
+            return
+        out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), bn, K, dtype,
+                      bias=dev_bf16(bias))
+        lin = bq.linear(dev_bf16(xb), dev_u8(qw), dev_f32(sw), bn, K, dtype, bias=dev_bf16(bias))
+        torch.cuda.synchronize()
+    finally:
+        bq.set_path(bq.PATH_AUTO)
+    bq.check_device_status()
+    ref = oracle.gemm(qa, sa, qw, sw, bn, K, dtype, bias_bf16=bias)
+    assert_gemm_close(out, ref, f"one scale block along K, M={M} N={N} K={K} bn={bn}")
+    assert_gemm_close(lin, ref, "bq_linear, one scale block along K")

@@ -22,9 +22,12 @@
 //               registers (scalar FADD/FFMA: measured faster here than the
 //               packed f32x2 forms), frees the buffer, and
 //               after the last K-block adds the bias and stores bf16.
+//   registers   setmaxnreg moves registers from the control warpgroup (56
+//               each) to the epilogue (104 each): no spills in the
+//               promotion loop (+5% INT8, +3% FP8 measured).
 // INT8 promotion without the int->float conversion unit: since
 // |P_kb| <= 128 * 128 * 128 < 2^22, the integer sum P_kb + 0x4B400000 (an
-// integer add on the ALU pipe) has the bits of the float 12582912 + P_kb
+// integer add) has the bits of the float 12582912 + P_kb
 // exactly, so one FADD recovers P_kb exactly and one FFMA promotes it (FMA
 // pipe).
 // A tile scheduler walks (expert, m-block, n-block) tiles; a dense problem is
@@ -66,6 +69,16 @@ using tc::sm_count;
 using tc::encode_fn;
 constexpr int kThreads = 640;        // 20 warps: A producer, MMA, W producer, idle, 16 epilogue
 constexpr int kEpiWarps = 16;
+// Register split (setmaxnreg): the control warpgroup (warps 0-3) gives up
+// registers, the four epilogue warpgroups take them, so that 64 fp32
+// accumulators and a 16-column TMEM chunk live in registers without spills.
+// The epilogue warpgroups' increase waits until the control warpgroup has
+// released enough: the split must fit the registers the CTA launched with,
+// which launch_typed checks against the compiled kernel before launching.
+constexpr int kCtrlRegs = 56;
+constexpr int kEpiRegs = 104;
+constexpr int kSplitRegs = 128 * kCtrlRegs + 32 * kEpiWarps * kEpiRegs;   // 60416
+static_assert(kSplitRegs <= 65536, "register split exceeds the SM's register file");
 // TMEM accumulators of BN columns: all 512 columns (4 x 128 or 2 x 256)
 template <int BN>
 constexpr int tbufs() { return 512 / BN; }
@@ -132,6 +145,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t tmem_base = *tmem_slot;
   const int total = tp_s[E];
 
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kCtrlRegs) : "memory");
   if (warp == 0 || warp == 2) {
     // ---------------- TMA producers: warp 0 the A tiles, warp 2 the W tiles
     // (one issuing thread sustains only part of the L2->SMEM rate a K-block
@@ -228,7 +243,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       while (!mbar_try_wait(smem_u32(&drain[0]), 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kEpiRegs) : "memory");
+  {
     // ---------------- epilogue ----------------
     constexpr int CW = BN / 4;                     // columns per epilogue warp
     const int q = warp & 3;
@@ -365,6 +383,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
     }
   }
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -385,6 +404,12 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::kTotal);
     if (e != cudaSuccess) return e;
+    // the register split must fit what the CTA is launched with, or the
+    // epilogue warps' setmaxnreg.inc would never be satisfied
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * kThreads < kSplitRegs) return cudaErrorInvalidConfiguration;
     attr_set[dev] = true;
   }
   CUtensorMap tA, tB;

@@ -62,6 +62,8 @@ DECLS = {
     "bq_grouped_gemm_workspace_size": (_INT, [_I64, _I64, _I64, _I64, _I64, _I64, _INT, _SZP]),
     "bq_grouped_gemm": (_INT, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _I64, _I64,
                                _I64, _INT, _P, _I64, _P, _SZ, _P]),
+    "bq_grouped_gemm_silu_quant": (_INT, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64,
+                                          _I64, _I64, _INT, _P, _I64, _P, _P]),
     "bq_moe_silu_mul_quant": (_INT, [_P, _I64, _I64, _I64, _I64, _INT, _P, _I64, _P, _P, _P]),
     "bq_moe_combine": (_INT, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _I64, _P]),
 }
@@ -316,6 +318,29 @@ def grouped_gemm(qa, sa, offsets, qw, sw, block_n=128, block_k=128, n_seam=0, dt
                                  _ld(out), _opt(ws, "ws"), 0 if ws is None else ws.numel(),
                                  _P(_stream(qa.device))))
     return out
+
+
+def grouped_gemm_silu_quant(qa, sa, offsets, qw13, sw13, dtype=INT8, q=None, s=None):
+    """w13 grouped GEMM fused with silu(gate) * up and its 1 x 128 requantisation.
+
+    qw13 [E, 2I, K] codes (gate rows then up rows), sw13 [E, 2I/128, Kb].
+    Returns the codes q [R, I] and scales s [I/128, R] of h; raises BqError
+    (ERR_UNSUPPORTED) where only the unfused calls apply.
+    """
+    R, K = qa.shape
+    E, N2, _ = qw13.shape
+    I = N2 // 2
+    if q is None:
+        q = torch.empty(R, I, dtype=torch.uint8, device=qa.device)
+    if s is None:
+        s = torch.empty(cdiv(I, 128), R, dtype=torch.float32, device=qa.device)
+    assert qw13.is_contiguous() and sw13.is_contiguous()
+    _check(lib().bq_grouped_gemm_silu_quant(_cuda(qa, "qa"), _ld(qa), _cuda(sa, "sa"), R,
+                                            _cuda(offsets, "offsets"), E, _cuda(qw13, "qw13"),
+                                            _cuda(sw13, "sw13"), I, K, 128, 128, dtype,
+                                            _cuda(q, "q"), _ld(q), _cuda(s, "s"),
+                                            _P(_stream(qa.device))))
+    return q, s
 
 
 def moe_silu_mul_quant(y, I, group_k=128, dtype=INT8, want_h=False, q=None, s=None):

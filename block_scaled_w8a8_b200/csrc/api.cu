@@ -14,6 +14,7 @@
 #include "bq_internal.h"
 #include "gemm_decode.h"
 #include "gemm_paths.h"
+#include "gemm_tc.h"
 
 namespace {
 
@@ -444,6 +445,41 @@ bq_status bq_grouped_gemm(const void* qa, int64_t lda, const float* sa, int64_t 
   if (rc == bq::kRunUnsupported) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
   if (rc == bq::kRunAlignment) return fail(BQ_ERR_ALIGNMENT, "%s", why);
   return fail(BQ_ERR_CUDA, "%s", why);
+}
+
+bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* sa, int64_t R,
+                                     const int32_t* expert_offsets, int64_t E, const void* qw13,
+                                     const float* sw13, int64_t I, int64_t K, int64_t block_n,
+                                     int64_t block_k, int dtype, void* q, int64_t ldq, float* s,
+                                     void* stream) {
+  BQ_CHECK_ARG(I >= 0, "I must be >= 0");
+  bq_status st = check_gemm_shape(R, 2 * I, K, block_n, block_k, dtype);
+  if (st != BQ_OK) return st;
+  BQ_CHECK_ARG(E >= 1 && E <= 65535, "E must be in [1, 65535]");
+  BQ_CHECK_ARG(lda >= K && ldq >= I, "leading dimensions too small");
+  if (R == 0 || I == 0) return ok();
+  BQ_CHECK_ARG(q && s && expert_offsets, "q, s and expert_offsets must not be NULL");
+  BQ_CHECK_ARG(K == 0 || (qa && sa && qw13 && sw13), "qa, sa, qw13 and sw13 must not be NULL");
+  if (!(g_path == BQ_PATH_AUTO || g_path == BQ_PATH_TCGEN05 || g_path == BQ_PATH_TCGEN05_1CTA))
+    return fail(BQ_ERR_UNSUPPORTED, "the fused SiLU GEMM runs on the tensor-core path only");
+  const int64_t Kb = cdiv(K, block_k);
+  bq::GemmArgs a{};
+  a.qa = qa; a.lda = lda; a.sa = sa; a.sa_rows = R;
+  a.qw = qw13; a.ldw = K; a.sw = sw13;
+  a.M = R; a.N = 2 * I; a.K = K; a.bn = block_n; a.bk = block_k; a.seam = I;
+  a.Nbs = 2 * cdiv(I, block_n);
+  a.dtype = dtype; a.bias = nullptr; a.out = nullptr; a.ldo = 0;
+  a.offsets = expert_offsets; a.E = E;
+  a.w_expert_stride = 2 * I * K; a.sw_expert_stride = a.Nbs * Kb;
+  a.q_out = q; a.ldq = ldq; a.s_out = s;
+  char why[256] = "";
+  if (!bq::tc_silu_supported(a, why, sizeof(why))) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
+  unsigned* w = nullptr;
+  st = status_word(&w);
+  if (st != BQ_OK) return st;
+  a.status = w;
+  BQ_CHECK_CUDA(bq::launch_gemm_tc_silu(a, as_stream(stream)), "fused SiLU GEMM launch");
+  return ok();
 }
 
 bq_status bq_moe_silu_mul_quant(const void* y, int64_t ldy, int64_t R, int64_t I,

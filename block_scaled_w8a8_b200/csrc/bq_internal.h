@@ -40,6 +40,10 @@ struct GemmArgs {
   int64_t w_expert_stride;   // bytes between experts' codes (N*K)
   int64_t sw_expert_stride;  // floats between experts' scales (Nbs*Kb)
   unsigned* status;
+  // fused SiLU * up + requantisation output (tcgen05 path only): when q_out
+  // is set, out is unused and the kernel writes codes [M, seam] (row stride
+  // ldq) and scales [seam / 128][sa_rows]
+  void* q_out; int64_t ldq; float* s_out;
 };
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);

@@ -87,16 +87,18 @@ template <int BN, int S>
 struct Smem {
   static constexpr uint32_t kA = BM * BK, kB = BN * BK;
   static constexpr uint32_t kStages = S * (kA + kB);
-  static constexpr uint32_t kBars = (2 * S + 2 * tbufs<BN>() + 2) * 8;
+  static constexpr uint32_t kBars = (2 * S + 2 * tbufs<BN>() + 3) * 8;
   static constexpr uint32_t kMisc = 8 + 2 * (kMaxE + 1) * 4;
-  static constexpr uint32_t kTotal = 1024 + kStages + kBars + kMisc;
+  // SILU: group amax of each tile row from its four column warps, two tiles
+  static constexpr uint32_t kAmax = 2 * 4 * BM * 4;
+  static constexpr uint32_t kTotal = 1024 + kStages + kBars + kMisc + kAmax;
 };
 
 // ONEK: the scale grid has a single K-block (block_k >= K: per-token
 // activation scales, per-channel or per-row-block weight scales).  The MMAs
 // then accumulate a tile's whole K in TMEM and the epilogue promotes once per
 // tile, out = P * sa[m] * sw[n / block_n], instead of once per K-block.
-template <int DT, int BN, int S, bool ONEK>
+template <int DT, int BN, int S, bool ONEK, bool SILU>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcParams p) {
@@ -113,10 +115,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = bars + 2 * S + kTBufs;
   uint64_t* drain = bars + 2 * S + 2 * kTBufs;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kTBufs + 1);
+  uint64_t* xbar = bars + 2 * S + 2 * kTBufs + 1;   // SILU: amax exchange
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kTBufs + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* off_s = reinterpret_cast<int*>(tmem_slot + 2);
   int* tp_s = off_s + (kMaxE + 1);
+  float* amax_s = reinterpret_cast<float*>(smem + L::kStages + L::kBars + L::kMisc);
+  static_assert(!SILU || (BN == 256 && !ONEK), "the fused SiLU epilogue uses 128 x 256 tiles");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
@@ -131,6 +136,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(smem_u32(&tempty[b]), kEpiWarps);
     }
     mbar_init(smem_u32(&drain[0]), 1);
+    mbar_init(smem_u32(&xbar[0]), kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -173,6 +179,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (is_a) {
             mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kA);
             tma_load_2d(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, smem_u32(&full[stage]));
+          } else if (SILU) {
+            // 128 gate rows, then the 128 up rows of the same h columns: the
+            // MMA's N = 256 operand is the two boxes back to back
+            mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kB);
+            const int g_row = e * (int)p.N + nb * 128;
+            tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, g_row,
+                        smem_u32(&full[stage]));
+            tma_load_2d(smem_u32(sB + stage * L::kB + 128 * BK), &tmB, kb * BK,
+                        g_row + (int)p.seam, smem_u32(&full[stage]));
           } else {
             mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kB);
             tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, b_row, smem_u32(&full[stage]));
@@ -254,7 +269,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int rit = 32 * q + lane;                 // row inside the tile
     const uint32_t tcol = (uint32_t)(CW * half);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint32_t kcount = 0;
+    uint32_t kcount = 0, tcount = 0;
     int e_hint = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -302,6 +317,47 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
         ++kcount;
+      } else if constexpr (SILU) {
+        // gate columns [32 * half, +32) and the up columns [128 + 32 * half,
+        // +32) of the same h columns: h = silu(g) * u needs both in one thread
+        const int64_t swg = (int64_t)nb * p.Kb;                  // gate scale row
+        const int64_t swu = ((p.seam >> 7) + nb) * p.Kb;         // up scale row
+        float sa_next = row_ok ? p.sa[m] : 0.f;
+        float sg_next = __ldg(sw_e + swg), su_next = __ldg(sw_e + swu);
+        for (int kb = 0; kb < p.Kb; ++kb) {
+          const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
+          const float fg = sa_next * sg_next, fu = sa_next * su_next;
+          if (kb + 1 < p.Kb) {
+            sa_next = row_ok ? p.sa[(int64_t)(kb + 1) * p.sa_rows + m] : 0.f;
+            sg_next = __ldg(sw_e + swg + kb + 1);
+            su_next = __ldg(sw_e + swu + kb + 1);
+          }
+          if (!warp_wait(smem_u32(&tfull[buf]), tround & 1, abort_flag, p.status, 0x306u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tb = tmem_base + lane_base + buf * BN + 32u * (uint32_t)half;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tb + (c < 2 ? 16u * c : 128u + 16u * (c - 2)), r);
+            tmem_ld_wait();
+            if (c == 3) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
+            }
+            const float f = c < 2 ? fg : fu;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float x = DT == kInt8 ? __uint_as_float(r[i] + kMagicBits) - kMagic
+                                          : __uint_as_float(r[i]);
+              accf[16 * c + i] = fmaf(x, f, accf[16 * c + i]);
+            }
+          }
+          ++kcount;
+        }
       } else {
         float sa_next = row_ok ? p.sa[m] : 0.f;      // K-block 0
         float sw_next = n0 < p.N ? __ldg(sw_e + swrow) : 0.f;
@@ -350,6 +406,43 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       }
       if (!ok) break;
+      if constexpr (SILU) {
+        // h = bf16(silu(g) * u) from the bf16-rounded GEMM outputs (what the
+        // unfused path stores and reads back), then the 1 x 128 quantisation
+        // of h: the tile's 128 h columns are exactly one group of each row
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float g = bf16_bits_to_float(float_to_bf16_bits(accf[j]));
+          const float u = bf16_bits_to_float(float_to_bf16_bits(accf[32 + j]));
+          const float sg = __fdiv_rn(g, 1.0f + expf(-g));
+          accf[j] = bf16_bits_to_float(float_to_bf16_bits(sg * u));
+          amax = fmaxf(amax, fabsf(accf[j]));
+        }
+        // the row's group amax from its four column warps (double-buffered
+        // by tile parity: the wait of the next tile orders reuse)
+        float* ax = amax_s + (tcount & 1u) * (4 * BM);
+        ax[half * BM + rit] = amax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&xbar[0]));
+        if (!warp_wait(smem_u32(&xbar[0]), tcount & 1u, abort_flag, p.status, 0x307u)) {
+          ok = false;
+          break;
+        }
+        const float gmax = fmaxf(fmaxf(ax[rit], ax[BM + rit]), fmaxf(ax[2 * BM + rit], ax[3 * BM + rit]));
+        const float sc = group_scale<DT>(gmax);
+        if (row_ok) {
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = pack4_codes<DT>(accf + 4 * i, sc);
+          uint4* qrow = reinterpret_cast<uint4*>(p.q_out + m * p.ldq + (int64_t)nb * 128 + 32 * half);
+          qrow[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          qrow[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          if (half == 0) p.s_out[(int64_t)nb * p.sa_rows + m] = sc;
+        }
+        ++tcount;
+        continue;
+      }
       if (row_ok && n0 < p.N) {
         uint16_t* orow = p.out + m * p.ldo + n0;
         const bool full_n = n0 + CW <= p.N;
@@ -393,10 +486,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
-template <int DT, int BN, int S, bool ONEK>
+template <int DT, int BN, int S, bool ONEK, bool SILU = false>
 cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   using L = Smem<BN, S>;
-  auto kern = gemm_tc_kernel<DT, BN, S, ONEK>;
+  auto kern = gemm_tc_kernel<DT, BN, S, ONEK, SILU>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -414,7 +507,8 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   }
   CUtensorMap tA, tB;
   if (!make_tmap(&tA, a.qa, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.lda, BM) ||
-      !make_tmap(&tB, a.qw, (uint64_t)a.K, (uint64_t)(a.N * a.E), (uint64_t)a.ldw, BN))
+      !make_tmap(&tB, a.qw, (uint64_t)a.K, (uint64_t)(a.N * a.E), (uint64_t)a.ldw,
+                 SILU ? 128u : (uint32_t)BN))
     return cudaErrorInvalidValue;
   TcParams p;
   p.sa = a.sa; p.sa_rows = a.sa_rows;
@@ -426,8 +520,9 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   p.offsets = a.offsets; p.E = (int)a.E;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;
-  p.nblk = (int)((a.N + BN - 1) / BN);
+  p.nblk = SILU ? (int)(a.seam / 128) : (int)((a.N + BN - 1) / BN);
   p.status = a.status;
+  p.q_out = static_cast<uint8_t*>(a.q_out); p.ldq = a.ldq; p.s_out = a.s_out;
   const int64_t mblk_bound = (a.M + BM - 1) / BM + (a.offsets ? a.E : 0);
   const int64_t tiles_bound = mblk_bound * p.nblk;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles_bound, sm_count()));
@@ -456,6 +551,28 @@ bool tc_supported(const GemmArgs& a, char* why, size_t n) {
   if (a.M > INT32_MAX || a.N * a.E > INT32_MAX || a.K > INT32_MAX) return no("sizes exceed int32");
   if (!encode_fn()) return no("cuTensorMapEncodeTiled is unavailable");
   return true;
+}
+
+bool tc_silu_supported(const GemmArgs& a, char* why, size_t n) {
+  auto no = [&](const char* msg) {
+    if (why) snprintf(why, n, "fused SiLU path: %s", msg);
+    return false;
+  };
+  if (!(a.bn == 128 && a.bk == 128)) return no("needs block_n = block_k = 128");
+  if (a.seam < 128 || a.seam % 128 != 0 || a.N != 2 * a.seam)
+    return no("needs a gate/up weight [2I, K] with I a multiple of 128");
+  if (a.bias) return no("takes no bias");
+  if (a.ldq % 16 != 0 || (reinterpret_cast<uintptr_t>(a.q_out) & 15))
+    return no("the code output needs 16-byte aligned rows");
+  GemmArgs b = a;
+  b.q_out = nullptr;
+  return tc_supported(b, why, n);
+}
+
+cudaError_t launch_gemm_tc_silu(const GemmArgs& a, cudaStream_t st) {
+  if (a.M == 0 || a.seam == 0) return cudaSuccess;
+  if (a.dtype == kInt8) return launch_typed<kInt8, 256, 4, false, true>(a, st);
+  return launch_typed<kFp8, 256, 4, false, true>(a, st);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {

@@ -30,6 +30,9 @@ struct TcParams {
   uint16_t* out; int64_t ldo;
   int nblk;                                     // tile columns
   unsigned* status;
+  // fused SiLU * up + requantisation (gate/up weight, seam = I): codes of h
+  // [rows, I] (row stride ldq) and scales [I / 128][sa_rows] instead of out
+  uint8_t* q_out; int64_t ldq; float* s_out;
 };
 
 // Weight-scale row of output column n (block_n = 128).  A fused gate+up

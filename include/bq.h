@@ -289,6 +289,31 @@ bq_status bq_grouped_gemm(const void* qa, int64_t lda, const float* sa, int64_t 
                           int64_t block_k, int64_t n_seam, int dtype, void* out, int64_t ldo,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* The w13 grouped GEMM fused with the SiLU * up requantisation (block-wise
+ * INT8 page, section 5: the gate+up weight, then the activation quantisation
+ * of the down projection's input).  For each expert e and each row r in
+ * [expert_offsets[e], expert_offsets[e+1]):
+ *   y[r, :] = bf16(block-scaled GEMM of qa[r] against qw13[e])  (as bq_grouped_gemm
+ *             with n_seam = I: gate rows [0, I), up rows [I, 2I));
+ *   h[r, i] = bf16(silu(y[r, i]) * y[r, I + i])                  (as bq_moe_silu_mul_quant);
+ *   q[r, :], s[:, r] = the 1 x 128 quantisation of h[r, :]        (as bq_quant_act).
+ * y and h are never stored: the tensor-core epilogue holds a tile's gate and
+ * up columns in registers.  The codes and scales are bit-identical to
+ * bq_grouped_gemm followed by bq_moe_silu_mul_quant with group_k = 128.
+ * qa: codes [R, K] (row stride lda), sa: fp32 [ceil(K/128)][R];
+ * qw13: codes [E, 2I, K] (dense), sw13: fp32 [E][2I/128][ceil(K/128)];
+ * q: codes [R, I] (row stride ldq, a multiple of 16; q 16-byte aligned),
+ * s: fp32 [I/128][R].  Rows past expert_offsets[E] are left untouched.
+ * Needs block_n = block_k = 128, I a multiple of 128, and the tensor-core
+ * path (BQ_PATH_AUTO, BQ_PATH_TCGEN05 or BQ_PATH_TCGEN05_1CTA); otherwise
+ * BQ_ERR_UNSUPPORTED, and the caller runs the two unfused calls.  Needs no
+ * workspace. */
+bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* sa, int64_t R,
+                                     const int32_t* expert_offsets, int64_t E, const void* qw13,
+                                     const float* sw13, int64_t I, int64_t K, int64_t block_n,
+                                     int64_t block_k, int dtype, void* q, int64_t ldq, float* s,
+                                     void* stream);
+
 /* h = bf16(silu(y[r, i]) * y[r, I + i]) (gate then up, block-wise INT8
  * page section 5 "gate + up fused"; SiLU is the reading for a gate/up pair),
  * then the activation quantisation of h with 1 x group_k groups.

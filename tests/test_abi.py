@@ -122,6 +122,17 @@ def test_quant_and_moe_argument_errors_on_host(L):
                              fake, 64, None, 0, None) == bq.ERR_INVALID_ARG   # seam > N
     assert L.bq_moe_silu_mul_quant(fake, 100, 4, 64, 128, 0, fake, 64, fake, None, None) == \
         bq.ERR_INVALID_ARG                                                     # ldy < 2I
+    # fused w13 + SiLU requantisation: ldq < I, then I not a multiple of 128
+    assert L.bq_grouped_gemm_silu_quant(fake, 128, fake, 8, fake, 2, fake, fake, 256, 128, 128,
+                                        128, 0, fake, 128, fake, None) == bq.ERR_INVALID_ARG
+    st, msg = _err(L, L.bq_grouped_gemm_silu_quant(fake, 128, fake, 8, fake, 2, fake, fake, 192,
+                                                   128, 128, 128, 0, fake, 192, fake, None))
+    assert st == bq.ERR_UNSUPPORTED and "multiple of 128" in msg
+    st, msg = _err(L, L.bq_grouped_gemm_silu_quant(fake, 128, fake, 8, fake, 2, fake, fake, 256,
+                                                   128, 64, 128, 0, fake, 256, fake, None))
+    assert st == bq.ERR_UNSUPPORTED and "block_n = block_k = 128" in msg
+    assert L.bq_grouped_gemm_silu_quant(None, 128, None, 0, fake, 2, None, None, 256, 128, 128,
+                                        128, 0, None, 256, None, None) == bq.OK   # R = 0
     assert L.bq_moe_combine(fake, 64, fake, fake, 4, 0, 64, fake, 64, None) == \
         bq.ERR_INVALID_ARG
     assert L.bq_set_path(9) == bq.ERR_INVALID_ARG

@@ -112,7 +112,7 @@ def moe_layer():
     import bench
     bq = _bq()
     layer = bench.MoeLayer(bq, torch.device("cuda"))
-    layer.run()
+    layer.run(bench.MoeLayer.UNFUSED)
     torch.cuda.synchronize()
     bq.check_device_status()
     yield layer
@@ -222,3 +222,18 @@ def test_moe_combine_full_size(moe_layer):
     inv = L.inv.cpu().numpy()
     assert_combine_close(L.out, oracle.moe_combine(yb, inv, L.tw), yb, inv, L.tw)
     assert np.isfinite(bf16_values(L.out)).all()
+
+
+def test_moe_fused_w13_silu_requant_full_size(moe_layer):
+    """The fused w13 + silu * up + requantisation call gives, on the full
+    layer, the same codes and scales as the unfused calls (whose every stage
+    the tests above check against the oracle)."""
+    L = moe_layer
+    c = L.cfg
+    q = torch.empty_like(L.qh)
+    s = torch.empty_like(L.sh)
+    L.bq.grouped_gemm_silu_quant(L.qa, L.sa, L.off, L.q13, L.s13, c.dtype, q=q, s=s)
+    torch.cuda.synchronize()
+    L.bq.check_device_status()
+    assert torch.equal(q, L.qh), "fused codes differ from the unfused calls"
+    assert torch.equal(s.view(torch.int32), L.sh.view(torch.int32)), "fused scales differ"

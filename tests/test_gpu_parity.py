@@ -462,6 +462,92 @@ def test_grouped_gemm_tcgen05_vs_oracle(path, dtype):
     assert_gemm_close(y13, ref13, "tcgen05 grouped w13")
 
 
+# w13 grouped GEMM fused with silu(gate) * up and the 1 x 128 requantisation
+# (T, H, I, E, dtype, seed): ragged experts, K with a partial last block,
+# several 128-column h groups, and an FP8 case
+SILU_CASES = [(300, 384, 256, 8, INT8, 33), (300, 384, 256, 8, FP8, 34),
+              (1000, 208, 384, 5, INT8, 35), (50, 128, 128, 4, FP8, 36),
+              (700, 512, 640, 8, INT8, 37)]
+
+
+@pytest.mark.parametrize("T,H,I,E,dtype,seed", SILU_CASES)
+def test_fused_w13_silu_requant(T, H, I, E, dtype, seed):
+    p = moe_problem(T=T, H=H, I=I, E=E, dtype=dtype, seed=seed)
+    topk = p["topk"]
+    off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), E)
+    o_ref, p_ref, _ = oracle.moe_permute(p["ids"], E)
+    qa, sa = bq.moe_quant_gather(dev_bf16(p["x"]), perm, topk, 128, dtype)
+    q13, s13 = dev_u8(p["q13"]), dev_f32(p["s13"])
+    qf, sf = bq.grouped_gemm_silu_quant(qa, sa, off, q13, s13, dtype)
+    # the unfused calls: w13 output in bf16, then silu * up and requantisation
+    y13 = bq.grouped_gemm(qa, sa, off, q13, s13, 128, 128, n_seam=I, dtype=dtype)
+    qu, su, hu = bq.moe_silu_mul_quant(y13, I, 128, dtype, want_h=True)
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    assert torch.equal(qf, qu), "fused codes differ from the unfused calls"
+    assert torch.equal(sf.view(torch.int32), su.view(torch.int32)), "fused scales differ"
+    # h (fp32 silu * up of the w13 output, one bf16 rounding) is within one
+    # bf16 ulp of the oracle's; the codes of that h are the oracle's exactly
+    h_or = oracle.bf16_to_f64(oracle.silu_mul(host_bits(y13), I))
+    hv = bf16_values(hu)
+    assert (np.abs(hv - h_or) <= bf16_ulp(np.maximum(np.abs(hv), np.abs(h_or)))).all()
+    qh, sh = oracle.quant_act(host_bits(hu), 128, dtype)
+    assert_codes_equal(qf, qh, "fused codes vs oracle quantisation of h")
+    assert_scales_equal(sf, sh, "fused scales vs oracle quantisation of h")
+    # the whole chain in the oracle (its own w13 GEMM): h agrees to the GEMM's
+    # tolerance, so the dequantised codes agree to within one code step
+    qx, sx = oracle.quant_act(p["x"], 128, dtype)
+    rows = p_ref // topk
+    ref13 = oracle.grouped_gemm(qx[rows], sx[rows], o_ref, p["q13"], p["s13"], 128, 128, dtype,
+                                seam=I)
+    h_ref = oracle.bf16_to_f64(oracle.silu_mul(oracle.bf16_from_f64(ref13), I))
+    deq = oracle.code_values(qf.cpu().numpy(), dtype) * np.repeat(sf.cpu().numpy().T, 128,
+                                                                    axis=1)[:, :I]
+    step = np.repeat(sf.cpu().numpy().T, 128, axis=1)[:, :I]
+    hmax = np.repeat(np.abs(h_ref).reshape(-1, I // 128, 128).max(axis=2), 128, axis=1)
+    if dtype == INT8:
+        tol = 0.5 * step + 2.0 ** -6 * hmax          # half a code + h within the GEMM's error
+    else:
+        tol = 2.0 ** -4 * np.abs(h_ref) + 2.0 ** -9 * step + 2.0 ** -6 * hmax
+    d = np.abs(deq - h_ref)
+    assert (d <= tol).all(), f"max excess {(d - tol).max()}"
+
+
+def test_fused_w13_silu_requant_rows_past_offsets_and_paths():
+    p = moe_problem(T=50, H=128, I=256, E=4, seed=38)
+    off = np.array([0, 10, 10, 30, 60], np.int32)     # 60 of the 100 rows routed
+    R, I = 100, 256
+    qa = torch.from_numpy(np.random.default_rng(5).integers(-127, 128, (R, 128)).astype(np.int8)
+                          .view(np.uint8)).cuda()
+    sa = torch.full((1, R), 0.01, dtype=torch.float32, device="cuda")
+    q = torch.full((R, I), 0x5A, dtype=torch.uint8, device="cuda")
+    s = torch.full((2, R), -1.0, dtype=torch.float32, device="cuda")
+    bq.grouped_gemm_silu_quant(qa, sa, dev_i32(off), dev_u8(p["q13"]), dev_f32(p["s13"]), INT8,
+                               q=q, s=s)
+    torch.cuda.synchronize()
+    assert (q[60:] == 0x5A).all() and (s[:, 60:] == -1.0).all()
+    y = bq.grouped_gemm(qa, sa, dev_i32(off), dev_u8(p["q13"]), dev_f32(p["s13"]), 128, 128,
+                        n_seam=I, dtype=INT8)
+    qu, su = bq.moe_silu_mul_quant(y[:60].contiguous(), I, 128, INT8)
+    assert torch.equal(q[:60], qu) and torch.equal(s[:, :60], su)
+    # TMA rows must be multiples of 16 bytes (K = 200 is not)
+    p2 = moe_problem(T=20, H=200, I=128, E=2, seed=39)
+    qa2 = torch.zeros(40, 200, dtype=torch.uint8, device="cuda")
+    sa2 = torch.ones(2, 40, dtype=torch.float32, device="cuda")
+    with pytest.raises(bq.BqError) as ei:
+        bq.grouped_gemm_silu_quant(qa2, sa2, dev_i32(np.array([0, 20, 40], np.int32)),
+                                   dev_u8(p2["q13"]), dev_f32(p2["s13"]), INT8)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+    # only the tensor-core path has the fused epilogue
+    for path in (bq.PATH_SIMT, bq.PATH_TCGEN05_2CTA):
+        bq.set_path(path)
+        with pytest.raises(bq.BqError) as ei:
+            bq.grouped_gemm_silu_quant(qa, sa, dev_i32(off), dev_u8(p["q13"]),
+                                       dev_f32(p["s13"]), INT8)
+        assert ei.value.status == bq.ERR_UNSUPPORTED
+    bq.set_path(bq.PATH_AUTO)
+
+
 @pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
 def test_grouped_gemm_leaves_rows_past_offsets_untouched(path):
     p = moe_problem(T=50, H=128, I=128, E=4)

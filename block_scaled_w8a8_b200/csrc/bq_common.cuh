@@ -45,6 +45,19 @@ __device__ __forceinline__ int int8_code(float x, float s) {
   return max(-128, min(127, r));
 }
 
+// INT8 code of x for scale s > 0 from rs = 1/s (correctly rounded), equal to
+// int8_code(x, s): for |x/s| < 128, q1 = fl(x * rs) is within 2^-16 of the
+// exact quotient and the IEEE quotient within 2^-18, so the two lie on the same
+// side of every rounding boundary n + 1/2 unless q1 is within 2^-13 of one;
+// there the IEEE division decides.  Larger |x/s| clamp either way.
+__device__ __forceinline__ int int8_code_recip(float x, float s, float rs) {
+  const float q1 = x * rs;
+  const float fr = q1 - floorf(q1);
+  if (fabsf(q1) < 128.0f && fabsf(fr - 0.5f) > 0x1p-13f)
+    return max(-128, min(127, __float2int_rn(q1)));
+  return int8_code(x, s);
+}
+
 // Two e4m3 codes (lo = x0, hi = x1) for scale s > 0, packed in 16 bits.
 __device__ __forceinline__ uint32_t e4m3x2_code(float x0, float x1, float s) {
   float c0 = __fdiv_rn(x0, s), c1 = __fdiv_rn(x1, s);
@@ -99,6 +112,15 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
 __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
   __nv_bfloat16 b = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&b);
+}
+
+// bf16 bits of silu(g) * u, silu(g) = g / (1 + exp(-g)) in fp32 with the
+// hardware exp2 and reciprocal (relative error ~1e-6, far below bf16's
+// half-ulp of 2^-9), rounded once to bf16.  Both the fused w13 epilogue and
+// the stand-alone SiLU kernel use this, so their h are identical.
+__device__ __forceinline__ uint16_t silu_mul_bf16(float g, float u) {
+  const float sg = __fdividef(g, 1.0f + __expf(-g));
+  return float_to_bf16_bits(sg * u);
 }
 
 }  // namespace bq

@@ -87,7 +87,7 @@ template <int BN, int S>
 struct Smem {
   static constexpr uint32_t kA = BM * BK, kB = BN * BK;
   static constexpr uint32_t kStages = S * (kA + kB);
-  static constexpr uint32_t kBars = (2 * S + 2 * tbufs<BN>() + 3) * 8;
+  static constexpr uint32_t kBars = (2 * S + 2 * tbufs<BN>() + 6) * 8;
   static constexpr uint32_t kMisc = 8 + 2 * (kMaxE + 1) * 4;
   // SILU: group amax of each tile row from its four column warps, two tiles
   static constexpr uint32_t kAmax = 2 * 4 * BM * 4;
@@ -115,8 +115,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = bars + 2 * S + kTBufs;
   uint64_t* drain = bars + 2 * S + 2 * kTBufs;
-  uint64_t* xbar = bars + 2 * S + 2 * kTBufs + 1;   // SILU: amax exchange
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kTBufs + 2);
+  uint64_t* xbar = bars + 2 * S + 2 * kTBufs + 1;   // SILU: amax exchange, per quadrant
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * kTBufs + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* off_s = reinterpret_cast<int*>(tmem_slot + 2);
   int* tp_s = off_s + (kMaxE + 1);
@@ -136,7 +136,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(smem_u32(&tempty[b]), kEpiWarps);
     }
     mbar_init(smem_u32(&drain[0]), 1);
-    mbar_init(smem_u32(&xbar[0]), kEpiWarps);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&xbar[i]), kEpiWarps / 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -415,17 +415,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int j = 0; j < 32; ++j) {
           const float g = bf16_bits_to_float(float_to_bf16_bits(accf[j]));
           const float u = bf16_bits_to_float(float_to_bf16_bits(accf[32 + j]));
-          const float sg = __fdiv_rn(g, 1.0f + expf(-g));
-          accf[j] = bf16_bits_to_float(float_to_bf16_bits(sg * u));
+          accf[j] = bf16_bits_to_float(silu_mul_bf16(g, u));
           amax = fmaxf(amax, fabsf(accf[j]));
         }
-        // the row's group amax from its four column warps (double-buffered
-        // by tile parity: the wait of the next tile orders reuse)
+        // the row's group amax from the four column warps of its TMEM lane
+        // quadrant (double-buffered by tile parity: the wait of the next tile
+        // orders reuse)
         float* ax = amax_s + (tcount & 1u) * (4 * BM);
         ax[half * BM + rit] = amax;
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&xbar[0]));
-        if (!warp_wait(smem_u32(&xbar[0]), tcount & 1u, abort_flag, p.status, 0x307u)) {
+        if (lane == 0) mbar_arrive(smem_u32(&xbar[q]));
+        if (!warp_wait(smem_u32(&xbar[q]), tcount & 1u, abort_flag, p.status, 0x307u)) {
           ok = false;
           break;
         }
@@ -433,8 +433,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const float sc = group_scale<DT>(gmax);
         if (row_ok) {
           uint32_t w[8];
+          if constexpr (DT == kInt8) {
+            // codes through the reciprocal of the scale, equal to the IEEE
+            // quotient's (int8_code_recip); a zero scale gives zero codes
+            const float rs = __frcp_rn(sc);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = pack4_codes<DT>(accf + 4 * i, sc);
+            for (int i = 0; i < 8; ++i) {
+              uint32_t ww = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int c = sc == 0.0f ? 0 : int8_code_recip(accf[4 * i + k], sc, rs);
+                ww |= (uint32_t)(uint8_t)(int8_t)c << (8 * k);
+              }
+              w[i] = ww;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack4_codes<DT>(accf + 4 * i, sc);
+          }
           uint4* qrow = reinterpret_cast<uint4*>(p.q_out + m * p.ldq + (int64_t)nb * 128 + 32 * half);
           qrow[0] = make_uint4(w[0], w[1], w[2], w[3]);
           qrow[1] = make_uint4(w[4], w[5], w[6], w[7]);

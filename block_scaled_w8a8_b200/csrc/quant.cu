@@ -67,9 +67,7 @@ struct RowSource {
       load4(up, k0, L, vec, u);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        // silu(g) = g / (1 + exp(-g)) in fp32, times u, rounded once to bf16
-        float sg = __fdiv_rn(g[i], 1.0f + expf(-g[i]));
-        uint16_t hb = float_to_bf16_bits(sg * u[i]);
+        const uint16_t hb = silu_mul_bf16(g[i], u[i]);
         v[i] = (k0 + i < L) ? bf16_bits_to_float(hb) : 0.0f;
       }
       if (h_out) {
@@ -214,9 +212,7 @@ quant_g128_kernel(const uint16_t* __restrict__ x, int64_t M_out, int64_t K, int6
           for (int h = 0; h < 2; ++h) {
             const float g = __uint_as_float(h ? (wa[e] & 0xFFFF0000u) : (wa[e] << 16));
             const float u = __uint_as_float(h ? (wb[e] & 0xFFFF0000u) : (wb[e] << 16));
-            // silu(g) = g / (1 + exp(-g)) in fp32, times u, rounded once to bf16
-            const float sg = __fdiv_rn(g, 1.0f + expf(-g));
-            hb[h] = float_to_bf16_bits(sg * u);
+            hb[h] = silu_mul_bf16(g, u);
             v[2 * e + h] = act[j] ? bf16_bits_to_float(hb[h]) : 0.0f;
           }
           hw[e] = (uint32_t)hb[0] | ((uint32_t)hb[1] << 16);

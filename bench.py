@@ -2,7 +2,7 @@
 """Throughput of the block-scaled W8A8 linear layer (libbq) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bq|reference]
-                    [--workload decode|prefill|fp8|moe] [--no-sub]
+                    [--workload decode|prefill|fp8|moe|perchannel] [--no-sub]
 
 Prints ONE JSON line.  The headline workload is the decode linear layer:
 INT8, N = K = 4096, [128,128] weight blocks, token counts M in {1, 8, 32, 64};
@@ -10,8 +10,10 @@ one step = for each M, the dynamic 1x128 activation quantisation followed by
 the block-scaled GEMM (bq_quant_act + bq_gemm, i.e. bq_linear).  Sixteen
 weight copies rotate (268 MB > the 126 MB L2), so every GEMM streams its
 weights from HBM.  `value` is whole-job algorithmic HBM bytes per second.
-Sub-workloads (prefill INT8 4096x14336x4096, FP8 e4m3 2048x4096x14336, and
-the INT8 MoE layer T=4096, E=8, top-2) report TOPS against the tensor roofline.
+Sub-workloads (prefill INT8 4096x14336x4096, FP8 e4m3 2048x4096x14336, the
+INT8 MoE layer T=4096, E=8, top-2 with the fused w13 + SiLU requantisation,
+and per-channel INT8 on the prefill shape) report TOPS against the tensor
+roofline.
 
 Multi-GPU: the layer shards over tokens with no exchange (replicas), so each
 rank runs the same per-rank work ("scaling": "weak"); time is the max over

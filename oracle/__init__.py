@@ -16,7 +16,10 @@ Sources are cited in ``bq_oracle.c``; in short:
     (section 4), MoE gate+up fused weights (section 5), int8 range (design
     rationale item 3);
   * SGLang quantization doc, "GEMM backends for FP4/FP8": blockwise FP8;
-  * "LLM quantization overview" page, FP8 section: e4m3 bit layout.
+  * "LLM quantization overview" page, FP8 section: e4m3 bit layout;
+  * MXFP8 (the doc's "MXFP8 dense linear"): the pages name it without
+    defining it; the reading is the microscaling format the name refers to
+    (32-element groups along K, power-of-two E8M0 scales, e4m3 elements).
 """
 from __future__ import annotations
 
@@ -78,6 +81,10 @@ def configure(lib):
     lib.bq_ref_silu_mul.restype = None
     lib.bq_ref_moe_combine.argtypes = [P, L, P, P, L, L, L, P]
     lib.bq_ref_moe_combine.restype = None
+    lib.bq_ref_mx_quant.argtypes = [P, L, L, L, P, L, P]
+    lib.bq_ref_mx_quant.restype = None
+    lib.bq_ref_mx_gemm.argtypes = [P, L, P, P, L, P, L, L, L, P, P]
+    lib.bq_ref_mx_gemm.restype = None
     return lib
 
 
@@ -297,4 +304,42 @@ def grouped_gemm(qa, sa, offsets, qw_e, sw_e, bn: int, bk: int, dtype: int, seam
         if r1 > r0:
             out[r0:r1] = gemm(qa[r0:r1], sa[r0:r1], qw_e[e], sw_e[e], bn, bk, dtype,
                               seam=seam)
+    return out
+
+
+# --------------------------------------------------------------------------
+# MXFP8 (32-element groups along K, E8M0 scales, e4m3 codes)
+# --------------------------------------------------------------------------
+
+MX_GROUP = 32
+
+
+def mx_quant(x: np.ndarray):
+    """MX quantisation of the rows of x, float values given as a float array
+    (bf16 or fp32 inputs converted exactly).  Returns (q uint8 [R, K] e4m3
+    codes, s uint8 [R, ceil(K/32)] E8M0 exponents, scale = 2^(s - 127))."""
+    lib = _load()
+    x = _c(x, np.float64)
+    R, K = x.shape
+    G = cdiv(K, MX_GROUP)
+    q = np.empty((R, K), dtype=np.uint8)
+    s = np.empty((R, G), dtype=np.uint8)
+    lib.bq_ref_mx_quant(_ptr(x), R, K, K, _ptr(q), K, _ptr(s))
+    return q, s
+
+
+def mx_gemm(qa, sa, qw, sw, bias_bf16=None):
+    """out64[m, n] = sum_g 2^(sa-127) 2^(sw-127) sum_{k in g} qa qw (+ bias), fp64."""
+    lib = _load()
+    qa = _c(qa, np.uint8)
+    qw = _c(qw, np.uint8)
+    sa = _c(sa, np.uint8)
+    sw = _c(sw, np.uint8)
+    M, K = qa.shape
+    N = qw.shape[0]
+    assert sa.shape == (M, cdiv(K, MX_GROUP)) and sw.shape == (N, cdiv(K, MX_GROUP))
+    b = None if bias_bf16 is None else _c(bias_bf16, np.uint16)
+    out = np.empty((M, N), dtype=np.float64)
+    lib.bq_ref_mx_gemm(_ptr(qa), K, _ptr(sa), _ptr(qw), K, _ptr(sw), M, N, K, _ptr(b),
+                       _ptr(out))
     return out

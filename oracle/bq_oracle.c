@@ -352,3 +352,80 @@ void bq_ref_moe_combine(const uint16_t* y, long ldy, const int32_t* inv_perm,
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP8 ([QDOC] "FP4/FP8 양자화용 GEMM 백엔드": MXFP8 dense linear)        */
+/* ------------------------------------------------------------------------ */
+/* The pages name the MXFP8 dense linear but do not define the format.
+ * Reading: the microscaling (MX) format the name refers to -- groups of 32
+ * consecutive elements along K share one scale 2^(E - 127) stored as an
+ * 8-bit exponent E (E8M0; 255 would be NaN and is never produced), elements
+ * are e4m3 codes.  The group's scale exponent is floor(log2(amax)) minus the
+ * largest exponent of an e4m3 normal (8), clamped to [-127, 127]; each
+ * element is x / 2^se (exact: a power-of-two scaling) converted to e4m3 by
+ * one round-to-nearest-even with saturation to +-448.  An all-zero group
+ * gets E = 0 and zero codes. */
+
+#define BQ_REF_MX_GROUP 32
+
+/* floor(log2(a)) for a finite a > 0, exactly (frexp: a = f * 2^e, f in [0.5, 1)). */
+static int floor_log2(double a) {
+    int e;
+    (void)frexp(a, &e);
+    return e - 1;
+}
+
+/* One group of L <= 32 values: returns the E8M0 byte, writes L codes. */
+static uint8_t mx_group(const double* x, long L, uint8_t* q) {
+    double amax = 0.0;
+    for (long i = 0; i < L; i++) {
+        double a = fabs(x[i]);
+        if (a > amax) amax = a;
+    }
+    int se = -127;
+    if (amax > 0.0) {
+        se = floor_log2(amax) - 8;
+        if (se < -127) se = -127;
+        if (se > 127) se = 127;
+    }
+    double inv = ldexp(1.0, -se);
+    for (long i = 0; i < L; i++) q[i] = bq_ref_e4m3_encode((float)(x[i] * inv));
+    return (uint8_t)(se + 127);
+}
+
+/* x: [R, K] doubles (exact copies of the bf16 or fp32 inputs), row stride ldx;
+ * q: [R, K] e4m3 codes (row stride ldq); s: [R, ceil(K/32)] E8M0 bytes
+ * row-major.  The last group of a row holds the remaining K mod 32 values. */
+void bq_ref_mx_quant(const double* x, long R, long K, long ldx, uint8_t* q, long ldq,
+                     uint8_t* s) {
+    long G = (K + BQ_REF_MX_GROUP - 1) / BQ_REF_MX_GROUP;
+    for (long r = 0; r < R; r++)
+        for (long g = 0; g < G; g++) {
+            long k0 = g * BQ_REF_MX_GROUP;
+            long L = (k0 + BQ_REF_MX_GROUP <= K) ? BQ_REF_MX_GROUP : K - k0;
+            s[r * G + g] = mx_group(x + r * ldx + k0, L, q + r * ldq + k0);
+        }
+}
+
+/* out[m, n] = sum_g 2^(sa[m,g]-127) * 2^(sw[n,g]-127) * sum_{k in g} qa[m,k] qw[n,k]
+ * (+ bias[n]) in fp64; out64 [M, N] row-major.  sa [M, G], sw [N, G] E8M0. */
+void bq_ref_mx_gemm(const uint8_t* qa, long lda, const uint8_t* sa, const uint8_t* qw,
+                    long ldw, const uint8_t* sw, long M, long N, long K,
+                    const uint16_t* bias, double* out) {
+    long G = (K + BQ_REF_MX_GROUP - 1) / BQ_REF_MX_GROUP;
+    for (long m = 0; m < M; m++)
+        for (long n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (long g = 0; g < G; g++) {
+                long k0 = g * BQ_REF_MX_GROUP;
+                long k1 = (k0 + BQ_REF_MX_GROUP <= K) ? k0 + BQ_REF_MX_GROUP : K;
+                double P = 0.0;
+                for (long k = k0; k < k1; k++)
+                    P += bq_ref_e4m3_decode(qa[m * lda + k]) * bq_ref_e4m3_decode(qw[n * ldw + k]);
+                acc += P * ldexp(1.0, (int)sa[m * G + g] - 127) *
+                       ldexp(1.0, (int)sw[n * G + g] - 127);
+            }
+            if (bias != NULL) acc += bq_ref_bf16_to_double(bias[n]);
+            out[m * N + n] = acc;
+        }
+}

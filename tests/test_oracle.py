@@ -436,3 +436,106 @@ def test_weight_bytes_arithmetic(golden):
     assert g["params"] * 1 / 1e9 == g["int8_GB"]
     overhead = 4.0 / (128 * 128)
     assert overhead < 3e-4
+
+
+# --------------------------------------------------------------------------
+# MXFP8: 32-element groups along K, E8M0 scales 2^(E-127), e4m3 codes
+# --------------------------------------------------------------------------
+
+def test_mx_quant_worked_example():
+    # amax 3 -> floor(log2 3) = 1 -> exponent 1 - 8 = -7 -> E = 120; the
+    # scaled values 384, -192, 32 are e4m3 codes 0 1111 100, 1 1110 100, 0 1100 000
+    x = np.zeros((1, 32))
+    x[0, :3] = [3.0, -1.5, 0.25]
+    q, s = oracle.mx_quant(x)
+    assert s.tolist() == [[120]]
+    assert [int(v) for v in q[0, :3]] == [0x7C, 0xF4, 0x60]
+    assert (q[0, 3:] == 0).all()
+
+
+def test_mx_quant_saturates_and_zero_group():
+    x = np.zeros((1, 96))
+    x[0, 32] = 500.0                      # floor(log2 500) = 8 -> E = 127, 500 -> 448
+    x[0, 33] = -0.5
+    q, s = oracle.mx_quant(x)
+    assert s.tolist() == [[0, 127, 0]]    # all-zero groups: E = 0, zero codes
+    assert q[0, 32] == 0x7E and oracle.e4m3_decode(np.array([q[0, 33]]))[0] == -0.5
+    assert (q[0, :32] == 0).all() and (q[0, 64:] == 0).all()
+
+
+@pytest.mark.parametrize("p", [-130, -126, -40, 0, 7, 8, 9, 60, 126])
+def test_mx_quant_scale_exponent_closed_form(p):
+    # a group whose amax is 1.5 * 2^p: E = clamp(p - 8, -127, 127) + 127, and
+    # every element that is an e4m3 value times 2^(p-8) comes back exactly
+    rng = np.random.default_rng(p + 200)
+    codes = rng.integers(0, 0x7F, 32).astype(np.uint8)
+    vals = oracle.e4m3_decode(codes) * np.where(rng.random(32) < 0.5, -1.0, 1.0)
+    vals[0] = 384.0                        # 1.5 * 2^8: sets the amax
+    x = np.ldexp(vals, p - 8)[None, :]
+    q, s = oracle.mx_quant(x)
+    se = max(-127, min(127, p - 8))
+    assert int(s[0, 0]) == se + 127
+    if se == p - 8:
+        assert np.array_equal(oracle.e4m3_decode(q[0]) * 2.0 ** se, x[0])
+
+
+def test_mx_quant_partial_last_group():
+    x = np.zeros((2, 40))
+    x[:, 32:] = [[1, 2, 3, 4, 5, 6, 7, 8], [0.5] * 8]   # 8 valid values
+    q, s = oracle.mx_quant(x)
+    assert s.shape == (2, 2)
+    assert s[0, 1] == 3 - 8 + 127 and s[1, 1] == -1 - 8 + 127     # amax 8 and 0.5
+    assert np.array_equal(oracle.e4m3_decode(q[0, 32:]) * 2.0 ** (s[0, 1] - 127.0),
+                          x[0, 32:])
+
+
+def test_mx_quant_matches_torch_float8_cast():
+    # the element rule is x / 2^se cast once to e4m3 with saturation; torch's
+    # float8_e4m3fn cast is round-to-nearest-even; magnitudes past 448 saturate
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(6, 128, generator=g, dtype=torch.float64) * 3.0)
+    q, s = oracle.mx_quant(x.numpy())
+    scale = torch.from_numpy(np.ldexp(1.0, s.astype(np.int64) - 127)).repeat_interleave(32, 1)
+    scaled = (x / scale).float()
+    assert scaled.abs().max() > 448       # the saturation is exercised
+    ref = scaled.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+
+
+def test_mx_gemm_unit_scales_is_a_matmul():
+    # E = 127 everywhere (scale 1): out = decoded A @ decoded W^T (BLAS fp64)
+    rng = np.random.default_rng(9)
+    qa = rng.integers(0, 256, (5, 96)).astype(np.uint8)
+    qw = rng.integers(0, 256, (7, 96)).astype(np.uint8)
+    qa[(qa & 0x7F) == 0x7F] = 0          # no NaN codes
+    qw[(qw & 0x7F) == 0x7F] = 0
+    sa = np.full((5, 3), 127, np.uint8)
+    sw = np.full((7, 3), 127, np.uint8)
+    ref = oracle.e4m3_decode(qa) @ oracle.e4m3_decode(qw).T
+    assert np.array_equal(oracle.mx_gemm(qa, sa, qw, sw), ref)
+
+
+def test_mx_gemm_scales_are_powers_of_two_per_group():
+    # brute force: dequantise every element with its own group's scale and
+    # contract in a different order (numpy einsum over dequantised matrices)
+    rng = np.random.default_rng(11)
+    M, N, K = 4, 6, 100
+    qa = rng.integers(0, 0x7E, (M, K)).astype(np.uint8) | (rng.integers(0, 2, (M, K)) << 7).astype(np.uint8)
+    qw = rng.integers(0, 0x7E, (N, K)).astype(np.uint8)
+    sa = rng.integers(110, 140, (M, 4)).astype(np.uint8)
+    sw = rng.integers(110, 140, (N, 4)).astype(np.uint8)
+    bias = oracle.bf16_from_f64(rng.normal(0, 1, N))
+    ka = np.ldexp(1.0, np.repeat(sa.astype(np.int64) - 127, 32, 1)[:, :K])
+    kw = np.ldexp(1.0, np.repeat(sw.astype(np.int64) - 127, 32, 1)[:, :K])
+    A = oracle.e4m3_decode(qa) * ka
+    W = oracle.e4m3_decode(qw) * kw
+    ref = np.einsum("mk,nk->mn", A, W) + oracle.bf16_to_f64(bias)[None, :]
+    out = oracle.mx_gemm(qa, sa, qw, sw, bias)
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-300)
+    # doubling one row's scale (E + 1) doubles that row's contraction exactly
+    sa2 = sa.copy()
+    sa2[2, 1] += 1
+    d = oracle.mx_gemm(qa, sa2, qw, sw) - oracle.mx_gemm(qa, sa, qw, sw)
+    part = (A[2, 32:64][None, :] * W[:, 32:64]).sum(axis=1)
+    np.testing.assert_allclose(d[2], part, rtol=1e-12)
+    assert (d[[0, 1, 3]] == 0).all()

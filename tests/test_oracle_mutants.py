@@ -39,6 +39,13 @@ MUTANTS = {
     "silu_sign": ("g / (1.0 + exp(-g)) * u", "g / (1.0 + exp(g)) * u"),
     "combine_first_weight_only": ("(double)w[t * topk + j]", "(double)w[t * topk]"),
     "bias_dropped": ("if (bias) acc += bq_ref_bf16_to_double(bias[n]);", ""),
+    "mx_scale_exponent_off_by_one": ("se = floor_log2(amax) - 8;", "se = floor_log2(amax) - 7;"),
+    "mx_no_low_clamp": ("if (se < -127) se = -127;", ""),
+    "mx_weight_scale_inverted": ("ldexp(1.0, (int)sw[n * G + g] - 127)",
+                                 "ldexp(1.0, 127 - (int)sw[n * G + g])"),
+    "mx_bias_dropped": ("if (bias != NULL) acc += bq_ref_bf16_to_double(bias[n]);", ""),
+    "mx_act_scale_first_group_only": ("ldexp(1.0, (int)sa[m * G + g] - 127)",
+                                      "ldexp(1.0, (int)sa[m * G] - 127)"),
     "bf16_ties_up": ("else r = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;\n    double res",
                      "else r = f + 1.0;\n    double res"),
 }

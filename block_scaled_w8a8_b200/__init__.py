@@ -65,6 +65,10 @@ DECLS = {
     "bq_grouped_gemm_silu_quant": (_INT, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64,
                                           _I64, _I64, _INT, _P, _I64, _P, _P]),
     "bq_moe_silu_mul_quant": (_INT, [_P, _I64, _I64, _I64, _I64, _INT, _P, _I64, _P, _P, _P]),
+    "bq_mx_scale_bytes": (_INT, [_I64, _I64, _SZP]),
+    "bq_mx_quant_act": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
+    "bq_mx_quant_weight": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
+    "bq_mx_gemm": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _P, _I64, _P]),
     "bq_moe_combine": (_INT, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _I64, _P]),
 }
 
@@ -341,6 +345,47 @@ def grouped_gemm_silu_quant(qa, sa, offsets, qw13, sw13, dtype=INT8, q=None, s=N
                                             _cuda(q, "q"), _ld(q), _cuda(s, "s"),
                                             _P(_stream(qa.device))))
     return q, s
+
+
+def mx_scale_bytes(R, K):
+    n = ctypes.c_size_t(0)
+    _check(lib().bq_mx_scale_bytes(R, K, ctypes.byref(n)))
+    return n.value
+
+
+def _mx_quant(fn, x, q=None, sf=None):
+    R, K = x.shape
+    if q is None:
+        q = torch.empty(R, K, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(mx_scale_bytes(R, K), dtype=torch.uint8, device=x.device)
+    _check(fn(_cuda(x, "x"), R, K, _ld(x), _cuda(q, "q"), _ld(q), _cuda(sf, "sf"),
+              _P(_stream(x.device))))
+    return q, sf
+
+
+def mx_quant_act(x, q=None, sf=None):
+    """MXFP8 quantisation of bf16 activations [M, K]: (e4m3 codes, scale atoms)."""
+    assert x.dtype == torch.bfloat16
+    return _mx_quant(lib().bq_mx_quant_act, x, q, sf)
+
+
+def mx_quant_weight(w, q=None, sf=None):
+    """MXFP8 quantisation of fp32 weights [N, K]: (e4m3 codes, scale atoms)."""
+    assert w.dtype == torch.float32
+    return _mx_quant(lib().bq_mx_quant_weight, w, q, sf)
+
+
+def mx_gemm(qa, sfa, qw, sfw, bias=None, out=None):
+    """MXFP8 linear: bf16 out [M, N] from e4m3 codes and their scale atoms."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=qa.device)
+    _check(lib().bq_mx_gemm(_cuda(qa, "qa"), _ld(qa), _cuda(sfa, "sfa"), _cuda(qw, "qw"),
+                            _ld(qw), _cuda(sfw, "sfw"), M, N, K, _opt(bias, "bias"),
+                            _cuda(out, "out"), _ld(out), _P(_stream(qa.device))))
+    return out
 
 
 def moe_silu_mul_quant(y, I, group_k=128, dtype=INT8, want_h=False, q=None, s=None):

@@ -13,6 +13,7 @@
 #include "bq_common.cuh"
 #include "bq_internal.h"
 #include "gemm_decode.h"
+#include "gemm_mx.h"
 #include "gemm_paths.h"
 #include "gemm_tc.h"
 
@@ -479,6 +480,76 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
   if (st != BQ_OK) return st;
   a.status = w;
   BQ_CHECK_CUDA(bq::launch_gemm_tc_silu(a, as_stream(stream)), "fused SiLU GEMM launch");
+  return ok();
+}
+
+// ---------------- MXFP8 ----------------
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bq_status bq_mx_scale_bytes(int64_t R, int64_t K, size_t* bytes) {
+  BQ_CHECK_ARG(bytes, "bytes must not be NULL");
+  BQ_CHECK_ARG(R >= 0 && K >= 0, "R and K must be >= 0");
+  if (K % 128 != 0) return fail(BQ_ERR_UNSUPPORTED, "MXFP8 needs K a multiple of 128");
+  *bytes = bq::mx_scale_bytes(R, K);
+  return ok();
+}
+
+static bq_status mx_quant_check(const void* x, int64_t R, int64_t K, int64_t ldx, void* q,
+                                int64_t ldq, void* sf) {
+  BQ_CHECK_ARG(R >= 0 && K >= 0, "rows and K must be >= 0");
+  BQ_CHECK_ARG(ldx >= K && ldq >= K, "leading dimensions too small");
+  if (K % 128 != 0) return fail(BQ_ERR_UNSUPPORTED, "MXFP8 needs K a multiple of 128");
+  if (R == 0 || K == 0) return BQ_OK;
+  BQ_CHECK_ARG(x && q && sf, "x, q and sf must not be NULL");
+  if (ldq % 4 != 0 || (reinterpret_cast<uintptr_t>(q) & 3))
+    return fail(BQ_ERR_ALIGNMENT, "MXFP8 codes need 4-byte aligned rows");
+  return BQ_OK;
+}
+
+bq_status bq_mx_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q,
+                          int64_t ldq, void* sf, void* stream) {
+  bq_status st = mx_quant_check(x, M, K, ldx, q, ldq, sf);
+  if (st != BQ_OK || M == 0 || K == 0) return st == BQ_OK ? ok() : st;
+  BQ_CHECK_CUDA(bq::launch_mx_quant_act(x, M, K, ldx, q, ldq, sf, as_stream(stream)),
+                "mx_quant_act launch");
+  return ok();
+}
+
+bq_status bq_mx_quant_weight(const float* w, int64_t N, int64_t K, int64_t ldw, void* q,
+                             int64_t ldq, void* sf, void* stream) {
+  bq_status st = mx_quant_check(w, N, K, ldw, q, ldq, sf);
+  if (st != BQ_OK || N == 0 || K == 0) return st == BQ_OK ? ok() : st;
+  BQ_CHECK_CUDA(bq::launch_mx_quant_weight(w, N, K, ldw, q, ldq, sf, as_stream(stream)),
+                "mx_quant_weight launch");
+  return ok();
+}
+
+bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* qw, int64_t ldw,
+                     const void* sfw, int64_t M, int64_t N, int64_t K, const void* bias,
+                     void* out, int64_t ldo, void* stream) {
+  BQ_CHECK_ARG(M >= 0 && N >= 0 && K >= 0, "M, N and K must be >= 0");
+  BQ_CHECK_ARG(lda >= K && ldw >= K && ldo >= N, "leading dimensions too small");
+  if (K % 128 != 0 || K == 0)
+    return fail(BQ_ERR_UNSUPPORTED, "MXFP8 GEMM needs K a positive multiple of 128");
+  if (M == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(qa && sfa && qw && sfw && out, "qa, sfa, qw, sfw and out must not be NULL");
+  if (!(g_path == BQ_PATH_AUTO || g_path == BQ_PATH_TCGEN05 || g_path == BQ_PATH_TCGEN05_1CTA))
+    return fail(BQ_ERR_UNSUPPORTED, "the MXFP8 GEMM runs on the tensor-core path only");
+  if (lda % 16 != 0 || ldw % 16 != 0 || !aligned16(qa) || !aligned16(qw) || !aligned16(sfa) ||
+      !aligned16(sfw))
+    return fail(BQ_ERR_ALIGNMENT,
+                "MXFP8 GEMM: code rows and bases, and the scale arrays, must be 16-byte aligned");
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+    return fail(BQ_ERR_UNSUPPORTED, "sizes exceed int32");
+  unsigned* w = nullptr;
+  bq_status st = status_word(&w);
+  if (st != BQ_OK) return st;
+  bq::MxArgs a{};
+  a.qa = qa; a.lda = lda; a.sfa = sfa;
+  a.qw = qw; a.ldw = ldw; a.sfw = sfw;
+  a.M = M; a.N = N; a.K = K; a.bias = bias; a.out = out; a.ldo = ldo; a.status = w;
+  BQ_CHECK_CUDA(bq::launch_gemm_mx(a, as_stream(stream)), "MXFP8 GEMM launch");
   return ok();
 }
 

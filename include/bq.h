@@ -314,6 +314,47 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
                                      int64_t block_k, int dtype, void* q, int64_t ldq, float* s,
                                      void* stream);
 
+/* ---------------- MXFP8 dense linear ----------------
+ * The SGLang quantization doc ("GEMM backends for FP4/FP8") lists an MXFP8
+ * dense linear beside the blockwise FP8 GEMM but does not define the format;
+ * the reading here is the microscaling format the name refers to.  Groups of
+ * 32 consecutive elements along K share a scale 2^(E - 127), E an 8-bit
+ * exponent (E8M0); elements are e4m3 codes.  Quantisation of a group:
+ * se = clamp(floor(log2 amax) - 8, -127, 127), E = se + 127, code =
+ * e4m3_rne_satfinite(x * 2^-se); an all-zero group has E = 0 and zero codes.
+ * Scale arrays use the tensor-core layout: rows in blocks of 128 and K in
+ * blocks of 128 (4 groups); each (row block, K block) is one 512-byte atom,
+ * atoms row-block major; row r, group g sits at byte
+ * 16*(r%32) + 4*((r%128)/32) + g%4 of its atom.  Bytes of rows past the last
+ * row are never written nor used.  K must be a multiple of 128. */
+
+/* Bytes of the scale array of R rows: ceil(R/128) * (K/128) * 512.
+ * BQ_ERR_UNSUPPORTED if K is not a multiple of 128. */
+bq_status bq_mx_scale_bytes(int64_t R, int64_t K, size_t* bytes);
+
+/* MX quantisation of bf16 activations x [M, K] (row stride ldx) into e4m3
+ * codes q [M, K] (row stride ldq, 4-byte aligned rows) and the scale array
+ * sf (bq_mx_scale_bytes(M, K) bytes). */
+bq_status bq_mx_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q,
+                          int64_t ldq, void* sf, void* stream);
+
+/* The same rule for fp32 weights w [N, K] (offline; row stride ldw). */
+bq_status bq_mx_quant_weight(const float* w, int64_t N, int64_t K, int64_t ldw, void* q,
+                             int64_t ldq, void* sf, void* stream);
+
+/* out[m, n] = bf16( sum_g 2^(Ea[m,g]-127) * 2^(Ew[n,g]-127) * sum_{k in g} a[m,k]*w[n,k]
+ *                   + bias[n] ), fp32 accumulation on the block-scaled tensor
+ * cores (tcgen05.mma kind::mxf8f6f4.block_scale; the scales are applied
+ * inside the MMA).  qa e4m3 [M, K] (row stride lda), sfa its scale array;
+ * qw e4m3 [N, K] (row stride ldw), sfw its scale array; bias bf16 [N] or
+ * NULL; out bf16 [M, N] (row stride ldo).  Needs K a positive multiple of
+ * 128, lda and ldw multiples of 16, and 16-byte aligned qa, qw, sfa, sfw
+ * (else BQ_ERR_UNSUPPORTED / BQ_ERR_ALIGNMENT), and the tensor-core path
+ * (BQ_PATH_AUTO, BQ_PATH_TCGEN05 or BQ_PATH_TCGEN05_1CTA).  No workspace. */
+bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* qw, int64_t ldw,
+                     const void* sfw, int64_t M, int64_t N, int64_t K, const void* bias,
+                     void* out, int64_t ldo, void* stream);
+
 /* h = bf16(silu(y[r, i]) * y[r, I + i]) (gate then up, block-wise INT8
  * page section 5 "gate + up fused"; SiLU is the reading for a gate/up pair),
  * then the activation quantisation of h with 1 x group_k groups.

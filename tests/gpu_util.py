@@ -100,3 +100,24 @@ def assert_combine_close(out: torch.Tensor, ref_bits: np.ndarray, y_bits: np.nda
         i = tuple(np.argwhere(bad)[0])
         raise AssertionError(f"{what}: {int(bad.sum())} outputs beyond the fp32-sum bound; "
                              f"first at {i}: gpu {g[i]!r} oracle {r[i]!r} tol {tol[i]!r}")
+
+
+# MXFP8 scale arrays: the library's tensor-core layout <-> the oracle's rows
+def _mx_sf_index(R, K):
+    r = np.arange(R)[:, None]
+    g = np.arange(K // 32)[None, :]
+    return (((r // 128) * (K // 128) + g // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32)
+            + g % 4)
+
+
+def mx_sf_rows(sf: torch.Tensor, R: int, K: int) -> np.ndarray:
+    """Scale atoms (flat uint8 tensor) -> per-row exponents [R, K/32]."""
+    return sf.cpu().numpy().reshape(-1)[_mx_sf_index(R, K)]
+
+
+def mx_sf_atoms(s_rows: np.ndarray, K: int) -> np.ndarray:
+    """Per-row exponents [R, K/32] -> the library's scale atoms (pad rows 127)."""
+    R = s_rows.shape[0]
+    out = np.full(((R + 127) // 128) * (K // 128) * 512, 127, np.uint8)
+    out[_mx_sf_index(R, K)] = s_rows
+    return out

@@ -135,6 +135,13 @@ def test_quant_and_moe_argument_errors_on_host(L):
                                         128, 0, None, 256, None, None) == bq.OK   # R = 0
     assert L.bq_moe_combine(fake, 64, fake, fake, 4, 0, 64, fake, 64, None) == \
         bq.ERR_INVALID_ARG
+    # MXFP8: K must be a multiple of 128; ld too small; empty problems
+    assert L.bq_mx_quant_act(fake, 4, 96, 96, fake, 96, fake, None) == bq.ERR_UNSUPPORTED
+    assert L.bq_mx_quant_act(fake, 4, 128, 64, fake, 128, fake, None) == bq.ERR_INVALID_ARG
+    assert L.bq_mx_gemm(fake, 256, fake, fake, 256, fake, 4, 8, 200, None, fake, 8, None) == \
+        bq.ERR_UNSUPPORTED
+    assert L.bq_mx_gemm(None, 256, None, None, 256, None, 0, 8, 256, None, None, 8, None) == bq.OK
+    assert bq.mx_scale_bytes(300, 512) == 3 * 4 * 512
     assert L.bq_set_path(9) == bq.ERR_INVALID_ARG
     assert L.bq_set_path(7) == bq.ERR_INVALID_ARG
     assert L.bq_selftest_bounded_wait(0, None) == bq.ERR_INVALID_ARG

@@ -13,7 +13,8 @@ import bq_synth
 import oracle
 from gpu_util import (assert_codes_equal, assert_combine_close, assert_gemm_close,
                       assert_scales_equal, bf16_ulp,
-                      bf16_values, dev_bf16, dev_f32, dev_i32, dev_u8, host_bits)
+                      bf16_values, dev_bf16, dev_f32, dev_i32, dev_u8, host_bits,
+                      mx_sf_atoms, mx_sf_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -634,3 +635,69 @@ def test_one_scale_block_along_k(path, M, N, K, bn, dtype):
     ref = oracle.gemm(qa, sa, qw, sw, bn, K, dtype, bias_bf16=bias)
     assert_gemm_close(out, ref, f"one scale block along K, M={M} N={N} K={K} bn={bn}")
     assert_gemm_close(lin, ref, "bq_linear, one scale block along K")
+
+
+# --------------------------------------------------------------------------
+# MXFP8 dense linear (32-element groups, E8M0 scales, block-scaled MMA)
+# --------------------------------------------------------------------------
+
+MX_QUANT_SHAPES = [(1, 128), (7, 256), (130, 384), (300, 1024)]
+
+
+@pytest.mark.parametrize("M,K", MX_QUANT_SHAPES)
+def test_mx_quant_act_and_weight_exact(M, K):
+    xb = act_bits(M, K, 700 + M, max(1, K // 100), 30.0)
+    xb[0, :32] = 0                                   # an all-zero group
+    q, sf = bq.mx_quant_act(dev_bf16(xb))
+    w = bq_synth.weights(M, K, 0.02, 701 + K).numpy()
+    qw, sfw = bq.mx_quant_weight(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    qr, sr = oracle.mx_quant(oracle.bf16_to_f64(xb))
+    assert_codes_equal(q, qr, "MX activation codes")
+    assert np.array_equal(mx_sf_rows(sf, M, K), sr), "MX activation scales"
+    qwr, swr = oracle.mx_quant(w.astype(np.float64))
+    assert_codes_equal(qw, qwr, "MX weight codes")
+    assert np.array_equal(mx_sf_rows(sfw, M, K), swr), "MX weight scales"
+
+
+MX_GEMM_SHAPES = [(1, 256, 128), (16, 320, 256), (200, 300, 512), (513, 1000, 1024),
+                  (128, 512, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", MX_GEMM_SHAPES)
+def test_mx_gemm_vs_oracle(M, N, K):
+    # codes and scales from the oracle (independent of the GPU quantiser),
+    # with a spread of scale exponents
+    rng = np.random.default_rng(M + N + K)
+    xa = rng.normal(0, 1, (M, K)) * np.exp2(rng.integers(-6, 7, (M, 1)))
+    xw = rng.normal(0, 0.02, (N, K)) * np.exp2(rng.integers(-3, 4, (N, K // 32))).repeat(32, 1)
+    qa, sa = oracle.mx_quant(xa)
+    qw, sw = oracle.mx_quant(xw)
+    bias = oracle.bf16_from_f64(rng.normal(0, 0.5, N))
+    out = bq.mx_gemm(dev_u8(qa), dev_u8(mx_sf_atoms(sa, K)), dev_u8(qw),
+                     dev_u8(mx_sf_atoms(sw, K)), bias=dev_bf16(bias))
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    assert_gemm_close(out, oracle.mx_gemm(qa, sa, qw, sw, bias), f"MXFP8 {M}x{N}x{K}")
+
+
+def test_mx_linear_end_to_end_and_errors():
+    M, N, K = 96, 384, 640
+    xb = act_bits(M, K, 710, 6, 30.0)
+    w = bq_synth.weights(N, K, 0.02, 711).numpy()
+    qa, sfa = bq.mx_quant_act(dev_bf16(xb))
+    qw, sfw = bq.mx_quant_weight(torch.from_numpy(w).cuda())
+    out = bq.mx_gemm(qa, sfa, qw, sfw)
+    torch.cuda.synchronize()
+    qar, sar = oracle.mx_quant(oracle.bf16_to_f64(xb))
+    qwr, swr = oracle.mx_quant(w.astype(np.float64))
+    assert_gemm_close(out, oracle.mx_gemm(qar, sar, qwr, swr), "MXFP8 linear")
+    # K must be a multiple of 128; only the tensor-core path has the kernel
+    with pytest.raises(bq.BqError) as ei:
+        bq.mx_quant_act(dev_bf16(act_bits(4, 96, 712)))
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+    bq.set_path(bq.PATH_SIMT)
+    with pytest.raises(bq.BqError) as ei:
+        bq.mx_gemm(qa, sfa, qw, sfw)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+    bq.set_path(bq.PATH_AUTO)

@@ -2,7 +2,7 @@
 """Throughput of the block-scaled W8A8 linear layer (libbq) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bq|reference]
-                    [--workload decode|prefill|fp8|moe|perchannel] [--no-sub]
+                    [--workload decode|prefill|fp8|moe|perchannel|mxfp8] [--no-sub]
 
 Prints ONE JSON line.  The headline workload is the decode linear layer:
 INT8, N = K = 4096, [128,128] weight blocks, token counts M in {1, 8, 32, 64};
@@ -12,8 +12,8 @@ weight copies rotate (268 MB > the 126 MB L2), so every GEMM streams its
 weights from HBM.  `value` is whole-job algorithmic HBM bytes per second.
 Sub-workloads (prefill INT8 4096x14336x4096, FP8 e4m3 2048x4096x14336, the
 INT8 MoE layer T=4096, E=8, top-2 with the fused w13 + SiLU requantisation,
-and per-channel INT8 on the prefill shape) report TOPS against the tensor
-roofline.
+per-channel INT8 on the prefill shape, and the MXFP8 linear on the FP8
+shape) report TOPS against the tensor roofline.
 
 Multi-GPU: the layer shards over tokens with no exchange (replicas), so each
 rank runs the same per-rank work ("scaling": "weak"); time is the max over
@@ -335,10 +335,11 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
     dev = torch.device("cuda", torch.cuda.current_device())
     M, N, K = cfg.M, cfg.N, cfg.K
     bn, bk = cfg.block_n, cfg.block_k
+    mx = cfg.dtype == bq_synth.MXFP8
     wq, wsc = [], []
     for i in range(n_rot):
         w = bq_synth.weights(N, K, cfg.w_std, cfg.seed + 10 * i, device=dev)
-        q, s = quant_weights(w, cfg.dtype, bq, bn, bk)
+        q, s = bq.mx_quant_weight(w) if mx else quant_weights(w, cfg.dtype, bq, bn, bk)
         wq.append(q)
         wsc.append(s)
         del w
@@ -347,12 +348,20 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
     out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     Kb = cdiv(K, bk)
     qa = torch.empty(M, K, dtype=torch.uint8, device=dev)
-    sa = torch.empty(Kb, M, dtype=torch.float32, device=dev)
-    gws = bq.workspace(bq.gemm_workspace_size(M, N, K, bn, bk, cfg.dtype), dev)
+    if mx:
+        sa = torch.empty(bq.mx_scale_bytes(M, K), dtype=torch.uint8, device=dev)
+    else:
+        sa = torch.empty(Kb, M, dtype=torch.float32, device=dev)
+        gws = bq.workspace(bq.gemm_workspace_size(M, N, K, bn, bk, cfg.dtype), dev)
     torch.cuda.synchronize()
 
     def step(i, quant=True):
         def run():
+            if mx:
+                if quant:
+                    bq.mx_quant_act(xs[i], q=qa, sf=sa)
+                bq.mx_gemm(qa, sa, wq[i], wsc[i], out=out)
+                return
             if quant:
                 bq.quant_act(xs[i], bk, cfg.dtype, q=qa, s=sa)
             bq.gemm(qa, sa, wq[i], wsc[i], bn, bk, cfg.dtype, out=out, ws=gws)
@@ -369,7 +378,9 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
     del graphs, gemm_graphs
     return {"value": whole_job_rate(dist.world, args.steps, ops, t) / 1e12, "unit": "TOPS",
             "ms_per_step": 1e3 * t / args.steps,
-            "roofline": {"bound": "tensor", "kernel": "tcgen05 block-scaled GEMM",
+            "roofline": {"bound": "tensor",
+                         "kernel": ("tcgen05 mxf8f6f4.block_scale GEMM" if mx else
+                                    "tcgen05 block-scaled GEMM"),
                          "achieved": ach, "peak": peak, "unit": "TFLOP/s" if cfg.dtype else
                          "TOPS", "frac": ach / peak, "traffic": None,
                          "peak_source": "2 x measured bf16 burst (8-bit dense = 2x bf16)",
@@ -377,7 +388,7 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
             "clocks": clk.summary(),
             "config": {"workload": cfg.name, "M": M, "N": N, "K": K, "block": [bn, bk],
                        "l2": f"{n_rot} rotating weight/activation copies"},
-            "dtype": "fp8_e4m3" if cfg.dtype else "int8"}
+            "dtype": "mxfp8_e4m3" if mx else "fp8_e4m3" if cfg.dtype else "int8"}
 
 
 class MoeLayer:
@@ -572,7 +583,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bq", choices=["bq", "reference"])
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "prefill", "fp8", "moe", "perchannel"])
+                    choices=["decode", "prefill", "fp8", "moe", "perchannel", "mxfp8"])
     ap.add_argument("--no-sub", action="store_true", help="skip the sub-workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline leg")
     args = ap.parse_args()
@@ -596,10 +607,12 @@ def main():
             head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.FP8_LINEAR, 3)
         elif args.workload == "perchannel":
             head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.PER_CHANNEL, 3)
+        elif args.workload == "mxfp8":
+            head = bench_linear_big(args, dist, bq, peaks, stream, bq_synth.MX_LINEAR, 3)
         else:
             head = bench_moe(args, dist, bq, peaks, stream)
         if not args.no_sub:
-            for name in ("prefill", "fp8", "moe", "perchannel"):
+            for name in ("prefill", "fp8", "moe", "perchannel", "mxfp8"):
                 if name == args.workload:
                     continue
                 torch.cuda.empty_cache()
@@ -612,6 +625,9 @@ def main():
                 elif name == "perchannel":
                     subs[name] = bench_linear_big(args, dist, bq, peaks, stream,
                                                   bq_synth.PER_CHANNEL, 3)
+                elif name == "mxfp8":
+                    subs[name] = bench_linear_big(args, dist, bq, peaks, stream,
+                                                  bq_synth.MX_LINEAR, 3)
                 else:
                     subs[name] = bench_moe(args, dist, bq, peaks, stream)
     bq.check_device_status()

@@ -20,6 +20,8 @@ blockwise FP8 linear layers, restated as synthetic inputs):
            w13 [8, 28672, 4096], w2 [8, 4096, 14336] ~ N(0, 0.015); seed 7
   perchannel  the prefill shape with block_n = 1, block_k = K (per-token and
            per-channel scales); seed 8
+  mxfp8    the FP8 shape, MXFP8 (1 x 32 groups, E8M0 scales) on both operands;
+           W ~ N(0, 0.01); seed 9
 
 Generators use torch.Generator so that the same recipe runs on the CPU (for
 oracle comparisons) or directly on a CUDA device (for large benchmarks).
@@ -33,6 +35,7 @@ import torch
 
 INT8 = 0
 FP8 = 1
+MXFP8 = 2        # workload marker: 32-element E8M0-scaled e4m3 groups
 
 
 @dataclasses.dataclass(frozen=True)
@@ -82,6 +85,9 @@ MOE = MoE("moe_int8_t4096_h4096_i14336_e8_top2", 4096, 4096, 14336, 8, 2, 0.015,
 # and one per output channel (block_n = 1), on the prefill shape
 PER_CHANNEL = Linear("perchannel_int8_m4096_n14336_k4096", 4096, 14336, 4096, 0.015,
                      one_percent(4096), 30.0, INT8, 8, block_n=1, block_k=4096)
+# the MXFP8 dense linear on the FP8 shape (1 x 32 scale groups on both sides)
+MX_LINEAR = Linear("mxfp8_m2048_n4096_k14336", 2048, 4096, 14336, 0.01, 0, 1.0, MXFP8, 9,
+                   block_n=1, block_k=32)
 
 
 def _gen(seed: int, device) -> torch.Generator:

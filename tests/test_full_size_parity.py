@@ -4,6 +4,7 @@ launch configuration that bench.py times:
   decode linear INT8     M in {1, 8, 32, 64}, N = K = 4096        (bq_linear)
   prefill up-proj INT8   M = 4096, N = 14336, K = 4096           (bq_quant_act + bq_gemm)
   blockwise FP8 linear   M = 2048, N = 4096,  K = 14336          (bq_quant_act + bq_gemm)
+  MXFP8 linear           M = 2048, N = 4096,  K = 14336          (bq_mx_quant_act + bq_mx_gemm)
   block-INT8 MoE layer   T = 4096, H = 4096, I = 14336, E = 8, top-2 (bench.MoeLayer)
 
 Activation codes and scales are compared bit-exactly over the whole tensors;
@@ -22,7 +23,7 @@ import torch
 import bq_synth
 import oracle
 from gpu_util import (assert_codes_equal, assert_combine_close, assert_gemm_close,
-                      assert_scales_equal, bf16_values, host_bits)
+                      assert_scales_equal, bf16_values, host_bits, mx_sf_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -105,6 +106,31 @@ def test_big_linear_full_size(cfg):
     rows = np.unique(np.concatenate([rows, [127, 128, 255, 256]]))
     ref = oracle.gemm(qr[rows], sr[rows], qw.cpu().numpy(), sw.cpu().numpy(), 128, 128, dt)
     assert_gemm_close(out[torch.from_numpy(rows).cuda()], ref, f"{cfg.name} sampled rows")
+
+
+def test_mx_linear_full_size():
+    """The MXFP8 linear on the FP8 shape: activation and weight codes and scales
+    bit-exact over the whole tensors, GEMM outputs on sampled rows."""
+    bq = _bq()
+    cfg = bq_synth.MX_LINEAR
+    M, N, K = cfg.M, cfg.N, cfg.K
+    w = bq_synth.weights(N, K, cfg.w_std, cfg.seed, device="cuda")
+    qw, sfw = bq.mx_quant_weight(w)
+    x = bq_synth.activations(M, K, cfg.seed, cfg.n_outliers, cfg.outlier_scale, device="cuda")
+    q, sfa = bq.mx_quant_act(x)
+    out = bq.mx_gemm(q, sfa, qw, sfw)
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    qwr, swr = oracle.mx_quant(w.cpu().double().numpy())
+    del w
+    assert_codes_equal(qw, qwr, "MX weight codes")
+    assert np.array_equal(mx_sf_rows(sfw, N, K), swr), "MX weight scales"
+    qr, sr = oracle.mx_quant(oracle.bf16_to_f64(host_bits(x)))
+    assert_codes_equal(q, qr, "MX activation codes")
+    assert np.array_equal(mx_sf_rows(sfa, M, K), sr), "MX activation scales"
+    rows = np.unique(np.concatenate([_sample_rows(M, 4, cfg.seed), [127, 128]]))
+    ref = oracle.mx_gemm(qr[rows], sr[rows], qwr, swr)
+    assert_gemm_close(out[torch.from_numpy(rows).cuda()], ref, "MXFP8 sampled rows")
 
 
 @pytest.fixture(scope="module")

@@ -337,68 +337,112 @@ gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 // ---------------- MX quantisation ----------------
 
-// One warp quantises 128 consecutive elements of a row (4 groups of 32); lane
-// l holds elements 4l .. 4l + 3, so lanes 8g .. 8g + 7 form group g.
+// A warp quantises a chunk of 256 consecutive elements of a row (8 groups of
+// 32, or the last 128 of a row); lane l holds elements 8l .. 8l + 7, so
+// lanes 4g .. 4g + 3 form group g.  Each warp keeps two chunks in flight.
 template <typename T>
-__global__ void __launch_bounds__(256)
-mx_quant_kernel(const T* __restrict__ x, int64_t R, int64_t K, int64_t ldx, bool vec,
-                uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf) {
-  const int64_t kc = K / 128;
-  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (w >= R * kc) return;
-  const int lane = threadIdx.x & 31;
-  const int64_t r = w / kc, c = w - r * kc;
-  const int64_t k0 = c * 128 + 4 * lane;
-  const T* src = x + r * ldx + k0;
-  float v[4];
+__device__ __forceinline__ void mx_load8(const T* __restrict__ src, bool vec, bool valid,
+                                         float (&v)[8]) {
+  if (!valid) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    return;
+  }
   if constexpr (sizeof(T) == 2) {
     if (vec) {
-      const uint2 u = *reinterpret_cast<const uint2*>(src);
-      v[0] = __uint_as_float(u.x << 16);
-      v[1] = __uint_as_float(u.x & 0xFFFF0000u);
-      v[2] = __uint_as_float(u.y << 16);
-      v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
     } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = bf16_bits_to_float(src[i]);
+      for (int i = 0; i < 8; ++i) v[i] = bf16_bits_to_float(src[i]);
     }
   } else {
     if (vec) {
-      const float4 u = *reinterpret_cast<const float4*>(src);
-      v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+      const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = src[i];
+      for (int i = 0; i < 8; ++i) v[i] = src[i];
     }
   }
-  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+}
+
+__device__ __forceinline__ void mx_finish8(const float (&v)[8], int64_t r, int64_t k0, bool valid,
+                                           int64_t K, uint8_t* __restrict__ q, int64_t ldq,
+                                           uint8_t* __restrict__ sf, int lane) {
+  float amax = 0.f;
 #pragma unroll
-  for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  if (!valid) return;
   // floor(log2 amax) is the unbiased exponent of a normal amax; a zero or
   // subnormal amax clamps to the smallest scale
   const int ef = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
   const int se = (ef == 0) ? -127 : max(-127, min(127, ef - 127 - 8));
   const float inv = __uint_as_float((uint32_t)(127 - se) << 23);   // 2^-se, exact
-  unsigned short lo, hi;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(v[1] * inv), "f"(v[0] * inv));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(v[3] * inv), "f"(v[2] * inv));
-  *reinterpret_cast<uint32_t*>(q + r * ldq + k0) = (uint32_t)lo | ((uint32_t)hi << 16);
-  if ((lane & 7) == 0) {
-    const int g = lane >> 3;
-    const int64_t atom = (r / 128) * kc + c;
-    sf[atom * kAtom + 16 * (r % 32) + 4 * ((r % 128) / 32) + g] = (uint8_t)(se + 127);
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    unsigned short lo, hi;
+    // the first source operand lands in the upper byte
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+        : "=h"(lo) : "f"(v[4 * h + 1] * inv), "f"(v[4 * h] * inv));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+        : "=h"(hi) : "f"(v[4 * h + 3] * inv), "f"(v[4 * h + 2] * inv));
+    w[h] = (uint32_t)lo | ((uint32_t)hi << 16);
+  }
+  uint32_t* dst = reinterpret_cast<uint32_t*>(q + r * ldq + k0);
+  dst[0] = w[0];
+  dst[1] = w[1];
+  if ((lane & 3) == 0) {
+    const int64_t gk = k0 / 32;                       // group index in the row
+    const int64_t atom = (r / 128) * (K / 128) + gk / 4;
+    sf[atom * kAtom + 16 * (r % 32) + 4 * ((r % 128) / 32) + gk % 4] = (uint8_t)(se + 127);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+mx_quant_kernel(const T* __restrict__ x, int64_t R, int64_t K, int64_t ldx, bool vec,
+                uint8_t* __restrict__ q, int64_t ldq, uint8_t* __restrict__ sf) {
+  const int64_t kc = (K + 255) / 256;                 // chunks per row
+  const int64_t total = R * kc;
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * 8;
+  for (int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); w < total; w += 2 * nw) {
+    const int64_t w2 = w + nw;
+    const int64_t r = w / kc, k0 = (w - r * kc) * 256 + 8 * lane;
+    const bool ok0 = k0 < K;
+    float a[8], b[8];
+    mx_load8(x + r * ldx + k0, vec, ok0, a);
+    int64_t r2 = 0, k2 = 0;
+    bool ok1 = false;
+    if (w2 < total) {
+      r2 = w2 / kc;
+      k2 = (w2 - r2 * kc) * 256 + 8 * lane;
+      ok1 = k2 < K;
+      mx_load8(x + r2 * ldx + k2, vec, ok1, b);
+    }
+    mx_finish8(a, r, k0, ok0, K, q, ldq, sf, lane);
+    if (w2 < total) mx_finish8(b, r2, k2, ok1, K, q, ldq, sf, lane);
   }
 }
 
 template <typename T>
 cudaError_t launch_mx_quant_t(const T* x, int64_t R, int64_t K, int64_t ldx, void* q,
                               int64_t ldq, void* sf, cudaStream_t st) {
-  const int64_t warps = R * (K / 128);
+  const int64_t warps = R * ((K + 255) / 256);
   if (warps == 0) return cudaSuccess;
-  const bool vec = (ldx * (int64_t)sizeof(T)) % (4 * sizeof(T)) == 0 &&
-                   (reinterpret_cast<uintptr_t>(x) % (4 * sizeof(T))) == 0;
-  const int64_t blocks = (warps + 7) / 8;
-  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  const bool vec = ldx % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+  const int64_t blocks = std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8);
   mx_quant_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(x, R, K, ldx, vec,
                                                         static_cast<uint8_t*>(q), ldq,
                                                         static_cast<uint8_t*>(sf));

@@ -284,18 +284,41 @@ def bench_decode(args, dist, bq, peaks, stream):
     clocks = clk.summary()
 
     # end to end through the public API with host buffers: H2D of the step's
-    # activations from pinned memory, bq_linear, D2H of the outputs
+    # activations from pinned memory, bq_linear, D2H of the outputs.  The four
+    # layers are independent, so the copies run on their own streams: every
+    # input goes up at the start of the step, each layer waits only for its
+    # own, and each output comes back as soon as its layer is done.
     hx = [x.cpu().pin_memory() for x in xs]
     ho = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in Ms]
     dx = [torch.empty_like(x, device=dev) for x in xs]
+    h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e(phase):
         def run():
+            comp = torch.cuda.current_stream()
+            start = torch.cuda.Event()
+            start.record(comp)
+            h2d_stream.wait_event(start)
+            d2h_stream.wait_event(start)
+            ready, done = [], []
+            with torch.cuda.stream(h2d_stream):
+                for j in range(len(Ms)):
+                    dx[j].copy_(hx[j], non_blocking=True)
+                    ready.append(torch.cuda.Event())
+                    ready[j].record(h2d_stream)
             for j, M in enumerate(Ms):
                 wi = (4 * phase + j) % NW
-                dx[j].copy_(hx[j], non_blocking=True)
+                comp.wait_event(ready[j])
                 bq.linear(dx[j], ws_q[wi], ws_s[wi], 128, 128, bq.INT8, out=outs[j], ws=lws)
-                ho[j].copy_(outs[j], non_blocking=True)
+                done.append(torch.cuda.Event())
+                done[j].record(comp)
+            with torch.cuda.stream(d2h_stream):
+                for j in range(len(Ms)):
+                    d2h_stream.wait_event(done[j])
+                    ho[j].copy_(outs[j], non_blocking=True)
+            fin = torch.cuda.Event()
+            fin.record(d2h_stream)
+            comp.wait_event(fin)
         return run
 
     e2e_graphs = [capture(e2e(p), stream) for p in range(phases)]

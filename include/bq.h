@@ -17,7 +17,8 @@
  *        gate and up projections fused, [E, 2I, H], scales
  *        [E, 2*ceil(I/bn), ceil(H/bk)].
  *  - SGLang "양자화 (Quantization)" doc, "FP4/FP8 양자화용 GEMM 백엔드":
- *      blockwise FP8 GEMM, the same contraction on e4m3 codes.
+ *      blockwise FP8 GEMM, the same contraction on e4m3 codes; the MXFP8
+ *      dense linear (format read as the microscaling one: see bq_mx_*).
  *  - "LLM 양자화 완전 정리 — FP8, AWQ, GPTQ, GGUF 차이와 선택법", FP8 section:
  *      e4m3 = 1 sign, 4 exponent, 3 mantissa bits.
  *
@@ -52,6 +53,8 @@
  *    (The pages do not fix this layout; K-block-major lets a GEMM tile read
  *    the scales of its rows for one K-block as one contiguous run.)
  *  - Weight scales are [Nb][Kb] row-major as on the block-wise INT8 page.
+ *  - The MXFP8 calls (bq_mx_*) keep their E8M0 scales in the tensor-core
+ *    atom layout described before bq_mx_scale_bytes.
  */
 #ifndef BQ_H_
 #define BQ_H_

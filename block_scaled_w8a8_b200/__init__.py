@@ -69,6 +69,9 @@ DECLS = {
     "bq_mx_quant_act": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "bq_mx_quant_weight": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "bq_mx_gemm": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _P, _I64, _P]),
+    "bq_mx_linear_workspace_size": (_INT, [_I64, _I64, _SZP]),
+    "bq_mx_linear": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _P, _SZ,
+                            _P]),
     "bq_moe_combine": (_INT, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _I64, _P]),
 }
 
@@ -385,6 +388,30 @@ def mx_gemm(qa, sfa, qw, sfw, bias=None, out=None):
     _check(lib().bq_mx_gemm(_cuda(qa, "qa"), _ld(qa), _cuda(sfa, "sfa"), _cuda(qw, "qw"),
                             _ld(qw), _cuda(sfw, "sfw"), M, N, K, _opt(bias, "bias"),
                             _cuda(out, "out"), _ld(out), _P(_stream(qa.device))))
+    return out
+
+
+def mx_linear_workspace_size(M, K):
+    n = ctypes.c_size_t(0)
+    _check(lib().bq_mx_linear_workspace_size(M, K, ctypes.byref(n)))
+    return n.value
+
+
+def mx_linear(x, qw, sfw, bias=None, out=None, ws=None):
+    """MXFP8 dense linear: bf16 x [M, K] -> bf16 [M, N] (activation MX
+    quantisation into the workspace, then the block-scaled MMA GEMM)."""
+    assert x.dtype == torch.bfloat16
+    M, K = x.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    nbytes = mx_linear_workspace_size(M, K)
+    if ws is None:
+        ws = workspace(nbytes, x.device)
+    _check(lib().bq_mx_linear(_cuda(x, "x"), _ld(x), M, K, _cuda(qw, "qw"), _ld(qw),
+                              _cuda(sfw, "sfw"), N, _opt(bias, "bias"), _cuda(out, "out"),
+                              _ld(out), _opt(ws, "ws"), 0 if ws is None else ws.numel(),
+                              _P(_stream(x.device))))
     return out
 
 

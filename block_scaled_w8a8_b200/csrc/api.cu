@@ -553,6 +553,45 @@ bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* q
   return ok();
 }
 
+static void mx_linear_layout(int64_t M, int64_t K, int64_t* ldq, size_t* sf_off,
+                             size_t* total) {
+  *ldq = (int64_t)round_up((size_t)K, 16);
+  *sf_off = round_up((size_t)(M * *ldq), 256);
+  *total = *sf_off + round_up(bq::mx_scale_bytes(M, K), 256);
+}
+
+bq_status bq_mx_linear_workspace_size(int64_t M, int64_t K, size_t* bytes) {
+  BQ_CHECK_ARG(bytes, "bytes must not be NULL");
+  BQ_CHECK_ARG(M >= 0 && K >= 0, "M and K must be >= 0");
+  if (K % 128 != 0) return fail(BQ_ERR_UNSUPPORTED, "MXFP8 needs K a multiple of 128");
+  int64_t ldq;
+  size_t so;
+  mx_linear_layout(M, K, &ldq, &so, bytes);
+  return ok();
+}
+
+bq_status bq_mx_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void* qw,
+                       int64_t ldw, const void* sfw, int64_t N, const void* bias, void* out,
+                       int64_t ldo, void* workspace, size_t workspace_bytes, void* stream) {
+  BQ_CHECK_ARG(M >= 0 && N >= 0 && K >= 0, "M, N and K must be >= 0");
+  BQ_CHECK_ARG(ldx >= K && ldw >= K && ldo >= N, "leading dimensions too small");
+  if (K % 128 != 0 || K == 0)
+    return fail(BQ_ERR_UNSUPPORTED, "MXFP8 linear needs K a positive multiple of 128");
+  if (M == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(x && qw && sfw && out, "x, qw, sfw and out must not be NULL");
+  int64_t ldq;
+  size_t so, need;
+  mx_linear_layout(M, K, &ldq, &so, &need);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(BQ_ERR_WORKSPACE, "bq_mx_linear needs %zu workspace bytes, got %zu", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(BQ_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  uint8_t* q = static_cast<uint8_t*>(workspace);
+  bq_status st = bq_mx_quant_act(x, M, K, ldx, q, ldq, q + so, stream);
+  if (st != BQ_OK) return st;
+  return bq_mx_gemm(q, ldq, q + so, qw, ldw, sfw, M, N, K, bias, out, ldo, stream);
+}
+
 bq_status bq_moe_silu_mul_quant(const void* y, int64_t ldy, int64_t R, int64_t I,
                                 int64_t group_k, int dtype, void* q, int64_t ldq, float* s,
                                 void* h_out, void* stream) {

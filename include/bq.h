@@ -358,6 +358,18 @@ bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* q
                      const void* sfw, int64_t M, int64_t N, int64_t K, const void* bias,
                      void* out, int64_t ldo, void* stream);
 
+/* Workspace for bq_mx_linear: the activation codes (rows padded to 16 bytes)
+ * and their scale atoms. */
+bq_status bq_mx_linear_workspace_size(int64_t M, int64_t K, size_t* bytes);
+
+/* The MXFP8 dense linear layer: bq_mx_quant_act of x (bf16 [M, K], row stride
+ * ldx) into the workspace, then bq_mx_gemm against qw / sfw (from
+ * bq_mx_quant_weight).  Same requirements as those two calls; workspace:
+ * bq_mx_linear_workspace_size bytes, 16-byte aligned, no initialisation. */
+bq_status bq_mx_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void* qw,
+                       int64_t ldw, const void* sfw, int64_t N, const void* bias, void* out,
+                       int64_t ldo, void* workspace, size_t workspace_bytes, void* stream);
+
 /* h = bf16(silu(y[r, i]) * y[r, I + i]) (gate then up, block-wise INT8
  * page section 5 "gate + up fused"; SiLU is the reading for a gate/up pair),
  * then the activation quantisation of h with 1 x group_k groups.

@@ -692,6 +692,12 @@ def test_mx_linear_end_to_end_and_errors():
     qar, sar = oracle.mx_quant(oracle.bf16_to_f64(xb))
     qwr, swr = oracle.mx_quant(w.astype(np.float64))
     assert_gemm_close(out, oracle.mx_gemm(qar, sar, qwr, swr), "MXFP8 linear")
+    # the one-call layer runs the same two kernels: identical output
+    bias = dev_bf16(oracle.bf16_from_f64(np.linspace(-1, 1, N)))
+    lin = bq.mx_linear(dev_bf16(xb), qw, sfw, bias=bias)
+    two = bq.mx_gemm(qa, sfa, qw, sfw, bias=bias)
+    torch.cuda.synchronize()
+    assert torch.equal(lin, two)
     # K must be a multiple of 128; only the tensor-core path has the kernel
     with pytest.raises(bq.BqError) as ei:
         bq.mx_quant_act(dev_bf16(act_bits(4, 96, 712)))

@@ -539,3 +539,29 @@ def test_mx_gemm_scales_are_powers_of_two_per_group():
     part = (A[2, 32:64][None, :] * W[:, 32:64]).sum(axis=1)
     np.testing.assert_allclose(d[2], part, rtol=1e-12)
     assert (d[[0, 1, 3]] == 0).all()
+
+
+def test_mx_quant_invariants_over_a_wide_range():
+    # whatever the magnitude: E never reaches 255 (NaN), no code is NaN
+    # (S.1111.111), and each element dequantises to within half an e4m3 step
+    # of its value (relative 2^-4 in the normal range, 2^-10 of the scale in
+    # the subnormal range), except where it saturates at 448 * scale
+    rng = np.random.default_rng(21)
+    R, K = 64, 256
+    x = rng.normal(0, 1, (R, K)) * np.exp2(rng.integers(-140, 121, (R, 1)))
+    x[5, :] = 0.0
+    x[6, 40] = -0.0
+    q, s = oracle.mx_quant(x)
+    assert s.max() <= 254
+    assert not np.any((q & 0x7F) == 0x7F)
+    scale = np.exp2(np.repeat(s.astype(np.float64) - 127, 32, axis=1))
+    deq = oracle.e4m3_decode(q) * scale
+    a = np.abs(x)
+    sat = a >= 448 * scale
+    err = np.abs(deq - x)
+    bound = np.maximum(2.0 ** -4 * a, 2.0 ** -10 * scale)
+    ok = (err <= bound) | sat
+    # elements below fp32's range after scaling are flushed by the float cast
+    tiny = a < 2.0 ** -149 * scale
+    assert np.all(ok | tiny)
+    assert np.all(np.abs(deq[sat]) == 448 * scale[sat])

@@ -707,3 +707,27 @@ def test_mx_linear_end_to_end_and_errors():
         bq.mx_gemm(qa, sfa, qw, sfw)
     assert ei.value.status == bq.ERR_UNSUPPORTED
     bq.set_path(bq.PATH_AUTO)
+
+
+def test_mx_gemm_narrow_n_and_strided_operands():
+    # N < 128 (one weight scale atom, half of the 256-wide tile unused) and
+    # codes read through row strides wider than K
+    rng = np.random.default_rng(77)
+    M, N, K = 3, 64, 256
+    qa, sa = oracle.mx_quant(rng.normal(0, 1, (M, K)))
+    qw, sw = oracle.mx_quant(rng.normal(0, 0.02, (N, K)))
+    out = bq.mx_gemm(dev_u8(qa), dev_u8(mx_sf_atoms(sa, K)), dev_u8(qw), dev_u8(mx_sf_atoms(sw, K)))
+    torch.cuda.synchronize()
+    assert_gemm_close(out, oracle.mx_gemm(qa, sa, qw, sw), "MXFP8 narrow N")
+    M, N, K = 150, 400, 384
+    qa, sa = oracle.mx_quant(rng.normal(0, 1, (M, K)))
+    qw, sw = oracle.mx_quant(rng.normal(0, 0.02, (N, K)))
+    wide_a = torch.zeros(M, K + 128, dtype=torch.uint8, device="cuda")
+    wide_w = torch.zeros(N, K + 64, dtype=torch.uint8, device="cuda")
+    wide_a[:, :K] = dev_u8(qa)
+    wide_w[:, :K] = dev_u8(qw)
+    out = bq.mx_gemm(wide_a[:, :K], dev_u8(mx_sf_atoms(sa, K)), wide_w[:, :K],
+                     dev_u8(mx_sf_atoms(sw, K)))
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    assert_gemm_close(out, oracle.mx_gemm(qa, sa, qw, sw), "MXFP8 strided operands")

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "bq.h"
 #include "bq_common.cuh"
@@ -59,10 +60,13 @@ __device__ unsigned g_bq_status_word;
 constexpr int kMaxDevices = 64;
 unsigned* g_status_ptr[kMaxDevices] = {};
 
+std::mutex g_status_mu;
+
 bq_status status_word(unsigned** out) {
   int dev = 0;
   BQ_CHECK_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(BQ_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_status_mu);
   if (!g_status_ptr[dev]) {
     void* p = nullptr;
     BQ_CHECK_CUDA(cudaGetSymbolAddress(&p, g_bq_status_word), "cudaGetSymbolAddress");
@@ -304,7 +308,7 @@ bq_status bq_gemm_decode_noalloc(const void* qa, int64_t lda, const float* sa, c
                 "bq_gemm_decode_noalloc holds %zu (use bq_gemm with a workspace)",
                 plan.ws_bytes, bq::kNoAllocScratchBytes);
   void* scratch = nullptr;
-  BQ_CHECK_CUDA(bq::noalloc_scratch(&scratch), "static scratch address");
+  BQ_CHECK_CUDA(bq::noalloc_scratch(&scratch, as_stream(stream)), "static scratch address");
   if (plan.ws_bytes > 0) {
     // arrival counters must start at zero; the partials need no clearing
     BQ_CHECK_CUDA(cudaMemsetAsync(scratch, 0, (size_t)plan.tiles * sizeof(unsigned),
@@ -553,10 +557,15 @@ bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* q
   return ok();
 }
 
-static void mx_linear_layout(int64_t M, int64_t K, int64_t* ldq, size_t* sf_off,
+// bq_mx_linear workspace: [64 KiB left untouched] [codes M x ldq] [scale atoms].
+// The first kDecodeCounterBytes are skipped, as in bq_linear, so that one
+// workspace can serve both calls: the decode GEMM keeps its arrival counters
+// there and needs them to stay zero.
+static void mx_linear_layout(int64_t M, int64_t K, int64_t* ldq, size_t* q_off, size_t* sf_off,
                              size_t* total) {
   *ldq = (int64_t)round_up((size_t)K, 16);
-  *sf_off = round_up((size_t)(M * *ldq), 256);
+  *q_off = bq::kDecodeCounterBytes;
+  *sf_off = *q_off + round_up((size_t)(M * *ldq), 256);
   *total = *sf_off + round_up(bq::mx_scale_bytes(M, K), 256);
 }
 
@@ -565,8 +574,8 @@ bq_status bq_mx_linear_workspace_size(int64_t M, int64_t K, size_t* bytes) {
   BQ_CHECK_ARG(M >= 0 && K >= 0, "M and K must be >= 0");
   if (K % 128 != 0) return fail(BQ_ERR_UNSUPPORTED, "MXFP8 needs K a multiple of 128");
   int64_t ldq;
-  size_t so;
-  mx_linear_layout(M, K, &ldq, &so, bytes);
+  size_t qo, so;
+  mx_linear_layout(M, K, &ldq, &qo, &so, bytes);
   return ok();
 }
 
@@ -580,16 +589,16 @@ bq_status bq_mx_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const v
   if (M == 0 || N == 0) return ok();
   BQ_CHECK_ARG(x && qw && sfw && out, "x, qw, sfw and out must not be NULL");
   int64_t ldq;
-  size_t so, need;
-  mx_linear_layout(M, K, &ldq, &so, &need);
+  size_t qo, so, need;
+  mx_linear_layout(M, K, &ldq, &qo, &so, &need);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(BQ_ERR_WORKSPACE, "bq_mx_linear needs %zu workspace bytes, got %zu", need,
                 workspace ? workspace_bytes : (size_t)0);
   if (!aligned16(workspace)) return fail(BQ_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
-  uint8_t* q = static_cast<uint8_t*>(workspace);
-  bq_status st = bq_mx_quant_act(x, M, K, ldx, q, ldq, q + so, stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  bq_status st = bq_mx_quant_act(x, M, K, ldx, base + qo, ldq, base + so, stream);
   if (st != BQ_OK) return st;
-  return bq_mx_gemm(q, ldq, q + so, qw, ldw, sfw, M, N, K, bias, out, ldo, stream);
+  return bq_mx_gemm(base + qo, ldq, base + so, qw, ldw, sfw, M, N, K, bias, out, ldo, stream);
 }
 
 bq_status bq_moe_silu_mul_quant(const void* y, int64_t ldy, int64_t R, int64_t I,

@@ -457,6 +457,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         named_bar(1, 128);
         if (et == 0) {
           const unsigned old = atomicAdd(&p.counters[tile], 1u);
+          // a counter that did not start at zero (the workspace's counter
+          // region was overwritten) would leave the tile unwritten: report it
+          if (old >= (unsigned)p.splits) record_status(p.status, kStatusBadInput, 0x406u);
           *last_flag = (old == (unsigned)(p.splits - 1)) ? 1 : 0;
         }
         named_bar(1, 128);
@@ -686,7 +689,7 @@ bool decode_supported(const GemmArgs& a, char* why, size_t n) {
 // process exits.  All calls share it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-cudaError_t noalloc_scratch(void** ptr) {
+cudaError_t noalloc_scratch(void** ptr, cudaStream_t st) {
   static std::mutex mu;
   static void* addr[kMaxScratchDevices] = {};
   int dev = 0;
@@ -694,9 +697,15 @@ cudaError_t noalloc_scratch(void** ptr) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    // The symbol's name is only a host-side handle: ask the runtime for the
-    // array's address on the current device, once per device.
+  // The symbol's name is only a host-side handle: ask the runtime for the
+  // array's address on the current device.  Outside stream capture the
+  // address is looked up again on every call, so a device reset (which
+  // reloads the module) cannot leave a stale pointer behind; a capturing
+  // stream reuses the address of the last uncaptured call on this device.
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  if (cs == cudaStreamCaptureStatusNone || addr[dev] == nullptr) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;

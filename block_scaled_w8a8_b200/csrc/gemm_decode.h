@@ -27,9 +27,9 @@ bool decode_supported(const GemmArgs& a, char* why, size_t n);
 // Fixed scratch of bq_gemm_decode_noalloc (counter region included).
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 constexpr int kMaxScratchDevices = 64;
-// Device address of that scratch on the current device (looked up on the
-// first call per device with cudaGetSymbolAddress).
-cudaError_t noalloc_scratch(void** ptr);
+// Device address of that scratch on the current device (cudaGetSymbolAddress;
+// looked up on every call made outside stream capture).
+cudaError_t noalloc_scratch(void** ptr, cudaStream_t st);
 
 // pdl: launch as a programmatic dependent of the preceding kernel (which must
 // not write the weights).  ws: zero-filled workspace of plan.ws_bytes.

@@ -194,7 +194,11 @@ bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_
  *   NULL when that size is 0).  Its first 64 KiB hold arrival counters: they
  *   must be zero before the workspace is first used, and every completed
  *   call leaves them zero again, whatever the shape, so one workspace can
- *   serve any sequence of calls.  The rest needs no initialisation.  Calls
+ *   serve any sequence of calls.  The rest needs no initialisation.  Every
+ *   libbq call that takes a workspace (bq_linear and bq_mx_linear included)
+ *   leaves these 64 KiB untouched, so one buffer can be shared by all of
+ *   them.  A counter found non-zero at a split's arrival is reported by
+ *   bq_check_device_status as invalid device-side input (site 0x406).  Calls
  *   sharing one workspace must not overlap on the GPU; after a call that
  *   reported a device error, zero the counter region again.
  * Block-wise INT8 page sections 2 and 4 (apply_w8a8_block_int8_linear with
@@ -217,8 +221,10 @@ bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, 
  * block_n = block_k = 128, 16-byte aligned operands and row strides, and a
  * split-K plan whose scratch fits in 16 MiB (e.g. M = 64 with N = K = 4096
  * fits; larger problems return BQ_ERR_UNSUPPORTED with the bytes needed).
- * The first call on each device looks up the array's device address; make
- * that first call before any stream capture.  Each call clears the counters
+ * Each call made outside stream capture looks up the array's device address
+ * (so a device reset cannot leave a stale address); a call made while its
+ * stream is capturing reuses the last address looked up on that device, so
+ * make the first call on each device before any stream capture.  Each call clears the counters
  * it uses.  All calls share the one array, so calls that overlap on the GPU
  * (different streams, or concurrent host threads) race and corrupt each
  * other's results: serialise them.  The pages have no counterpart to this
@@ -365,7 +371,9 @@ bq_status bq_mx_linear_workspace_size(int64_t M, int64_t K, size_t* bytes);
 /* The MXFP8 dense linear layer: bq_mx_quant_act of x (bf16 [M, K], row stride
  * ldx) into the workspace, then bq_mx_gemm against qw / sfw (from
  * bq_mx_quant_weight).  Same requirements as those two calls; workspace:
- * bq_mx_linear_workspace_size bytes, 16-byte aligned, no initialisation. */
+ * bq_mx_linear_workspace_size bytes, 16-byte aligned, no initialisation.
+ * The codes start 64 KiB into the workspace: its first 64 KiB are left
+ * untouched, so the same buffer can also serve bq_gemm / bq_linear. */
 bq_status bq_mx_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void* qw,
                        int64_t ldw, const void* sfw, int64_t N, const void* bias, void* out,
                        int64_t ldo, void* workspace, size_t workspace_bytes, void* stream);

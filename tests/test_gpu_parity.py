@@ -709,6 +709,39 @@ def test_mx_linear_end_to_end_and_errors():
     bq.set_path(bq.PATH_AUTO)
 
 
+def test_shared_workspace_survives_every_entry_point():
+    """One workspace buffer serves bq_mx_linear, bq_gemm and bq_linear in any
+    order: no call may leave bytes in the region where the decode GEMM keeps
+    its split-K arrival counters.  An MXFP8 linear (61 440 code bytes) runs
+    first on the binding's cached workspace, then decode GEMMs whose split
+    partials are reduced through that workspace, each against the oracle."""
+    M, N, K = 96, 384, 640
+    xb = act_bits(M, K, 720, 6, 30.0)
+    w = bq_synth.weights(N, K, 0.02, 721).numpy()
+    qw, sfw = bq.mx_quant_weight(torch.from_numpy(w).cuda())
+    x = dev_bf16(xb)
+    need = max(bq.mx_linear_workspace_size(M, K), bq.gemm_workspace_size(1, 640, 1008),
+               bq.linear_workspace_size(33, 1000, 2048))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    bq.mx_linear(x, qw, sfw, ws=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:65536].count_nonzero()) == 0, "bq_mx_linear wrote into the counter region"
+    for (Md, Nd, Kd), seed in (((1, 640, 1008), 722), ((33, 1000, 2048), 723)):
+        xd, qa, sa, qwd, swd, _ = make_problem(Md, Nd, Kd, 128, 128, INT8, seed)
+        ref = oracle.gemm(qa, sa, qwd, swd, 128, 128, INT8)
+        assert bq.gemm_workspace_size(Md, Nd, Kd) > 0, "shape must use the workspace"
+        out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qwd), dev_f32(swd), out=None, ws=ws)
+        lin = bq.linear(dev_bf16(xd), dev_u8(qwd), dev_f32(swd), ws=ws)
+        bq.mx_linear(x, qw, sfw, ws=ws)
+        again = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qwd), dev_f32(swd), ws=ws)
+        torch.cuda.synchronize()
+        bq.check_device_status()
+        assert_gemm_close(out, ref, f"decode after mx_linear {Md}x{Nd}x{Kd}")
+        assert_gemm_close(lin, ref, f"linear after decode {Md}x{Nd}x{Kd}")
+        assert torch.equal(out, again), "decode output depends on the call before it"
+        assert int(ws[:65536].count_nonzero()) == 0, "counters not left at zero"
+
+
 def test_mx_gemm_narrow_n_and_strided_operands():
     # N < 128 (one weight scale atom, half of the 256-wide tile unused) and
     # codes read through row strides wider than K

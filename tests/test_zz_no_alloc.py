@@ -74,6 +74,41 @@ def test_noalloc_matches_workspace_entry_point_twice(dtype, M, N, K):
         _close(out, ref, f"call {i} dtype={dtype} {M}x{N}x{K}")
 
 
+def test_noalloc_allocates_nothing_across_shapes_back_to_back():
+    """Two shapes with different tile counts, whose partials both go through
+    the fixed scratch, called alternately: each call clears the counters it
+    uses, and device memory stays exactly as free as before the calls."""
+    torch.cuda.set_device(0)
+    shapes = [(1, 640, 1008), (33, 1000, 2048)]
+    ops = [_operands(M, N, K, bq.INT8, 950 + M) for M, N, K in shapes]
+    refs, outs = [], []
+    bq.set_path(bq.PATH_DECODE)
+    try:
+        for (M, N, K), (qa, sa, qw, sw, bias) in zip(shapes, ops):
+            refs.append(bq.gemm(qa, sa, qw, sw, 128, 128, bq.INT8, bias=bias))
+    finally:
+        bq.set_path(bq.PATH_AUTO)
+    for (M, N, K) in shapes:
+        outs.append([torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+                     for _ in range(2)])
+    # the first call looks up the scratch's address; then measure
+    qa, sa, qw, sw, bias = ops[0]
+    assert _call_c_abi(qa, sa, qw, sw, bq.INT8, bias, outs[0][0]) == bq.OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for rep in range(2):
+        for i, (qa, sa, qw, sw, bias) in enumerate(ops):
+            assert _call_c_abi(qa, sa, qw, sw, bq.INT8, bias, outs[i][rep]) == bq.OK, \
+                bq.lib().bq_last_error_message()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    bq.check_device_status()
+    assert free1 == free0, f"device memory changed by {free0 - free1} bytes"
+    for i, (M, N, K) in enumerate(shapes):
+        for rep in range(2):
+            _close(outs[i][rep], refs[i], f"{M}x{N}x{K} call {rep}")
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     M, N, K = 128, 1920, 4096        # 15 weight tiles x 20 splits: ~19.7 MB of partials
     qa, sa, qw, sw, _ = _operands(M, N, K, bq.INT8, 7)

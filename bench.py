@@ -182,9 +182,11 @@ class Clocks:
             os.remove(self.path)
         except OSError:
             pass
-        loaded = [m for m in mhz if mx and m > 0.5 * mx] or mhz
-        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
-                "samples": len(mhz), "reasons": sorted(reasons)}
+        # every sample taken while the timed region ran counts: a clock stuck
+        # low must show in the median, not be filtered out
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "sm_min_mhz": min(mhz) if mhz else None, "samples": len(mhz),
+                "reasons": sorted(reasons)}
 
 
 # --------------------------------------------------------------------------
@@ -325,13 +327,16 @@ def bench_decode(args, dist, bq, peaks, stream):
     t_e2e = timed_graph_steps(e2e_graphs, args.steps, args.warmup, stream, dist)
 
     n = dist.world
-    traffic, traffic_src = load_traffic("gemm_decode.cu")
+    traffic, traffic_src = load_traffic("gemm_decode_cluster.cu")
     value = whole_job_rate(n, args.steps, step_bytes, t) / 1e9
     gemm_launch_s = t_gemm / (args.steps * len(Ms))
     achieved = gemm_bytes / len(Ms) / gemm_launch_s / 1e9
     res = {
         "value": value, "unit": "GB/s", "ms_per_step": 1e3 * t / args.steps,
-        "roofline": {"bound": "hbm", "kernel": "block-scaled GEMM (decode shapes)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "gemm_decode_cluster_kernel (block-scaled decode GEMM; four "
+                               "launches per step, consecutive launches overlapped by "
+                               "programmatic dependent launch)",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "traffic_source": traffic_src,
@@ -412,6 +417,34 @@ def bench_linear_big(args, dist, bq, peaks, stream, cfg, n_rot):
             "config": {"workload": cfg.name, "M": M, "N": N, "K": K, "block": [bn, bk],
                        "l2": f"{n_rot} rotating weight/activation copies"},
             "dtype": "mxfp8_e4m3" if mx else "fp8_e4m3" if cfg.dtype else "int8"}
+
+
+def bench_tiny(args, dist, bq, stream):
+    """Latency of the tiny block-wise INT8 linear layer (M = 16, N = 320,
+    K = 200: partial blocks, the CUDA-core path since K = 200 is not a
+    16-byte row), one bq_linear per call, 20 calls per graph replay."""
+    cfg = bq_synth.TINY
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = bq_synth.weights(cfg.N, cfg.K, cfg.w_std, cfg.seed, device=dev)
+    qw, sw = quant_weights(w, cfg.dtype, bq, cfg.block_n, cfg.block_k)
+    x = bq_synth.activations(cfg.M, cfg.K, cfg.seed, cfg.n_outliers, cfg.outlier_scale,
+                             device=dev)
+    out = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16, device=dev)
+    ws = bq.workspace(bq.linear_workspace_size(cfg.M, cfg.N, cfg.K), dev)
+    calls = 20
+
+    def run():
+        for _ in range(calls):
+            bq.linear(x, qw, sw, cfg.block_n, cfg.block_k, cfg.dtype, out=out, ws=ws)
+
+    g = [capture(run, stream)]
+    steps = max(3, args.steps // 4)
+    t = timed_graph_steps(g, steps, args.warmup, stream, dist)
+    del g
+    return {"value": 1e6 * t / (steps * calls), "unit": "us", "higher_is_better": False,
+            "config": {"workload": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K,
+                       "block": [cfg.block_n, cfg.block_k]},
+            "dtype": "int8", "note": "latency of one bq_linear call (quantiser + GEMM)"}
 
 
 class MoeLayer:
@@ -560,15 +593,171 @@ class OracleDecode:
         return time.perf_counter() - t0
 
 
-def cpu_baseline(seconds_target=15.0):
-    od = OracleDecode()
-    first = od.step()
+def host_info():
+    """Host cores and CPU model of the machine the CPU baseline runs on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count() or 1, "cpu_model": model}
+
+
+def _timed_reps(step, seconds_target):
+    first = step()
     reps = max(1, int(seconds_target / max(first, 1e-3)))
-    dt = sum(od.step() for _ in range(reps))
-    return {"value": reps * od.bytes_per_step / dt / 1e9, "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{reps} whole decode steps (M in 1,8,32,64; N = K = 4096) after one "
-                      f"untimed step; single-threaded C oracle; {dt:.1f} s"}
+    return reps, sum(step() for _ in range(reps))
+
+
+def cpu_baseline(seconds_target=8.0):
+    """The decode workload on the oracle: single-threaded (the plain build) and
+    on all host cores (the OpenMP build, rows split over threads)."""
+    import oracle
+    hi = host_info()
+    od = OracleDecode()
+    res = {}
+    for threads in (1, hi["nproc"]):
+        used = oracle.use_threads(threads)
+        try:
+            reps, dt = _timed_reps(od.step, seconds_target if threads == 1 else seconds_target / 2)
+        finally:
+            oracle.use_threads(1)
+        res[threads] = {"value": reps * od.bytes_per_step / dt / 1e9, "unit": "GB/s",
+                        "cores": used, "kind": "oracle",
+                        "sample": f"{reps} whole decode steps (M in 1,8,32,64; N = K = 4096) "
+                                  f"after one untimed step; C oracle on {used} thread(s); "
+                                  f"{dt:.1f} s"}
+    one, allc = res[1], res[hi["nproc"]]
+    return dict(allc, single_thread=one, host=hi)
+
+
+def cpu_baseline_linear(cfg, seconds_target=3.0):
+    """A bounded sample of a big linear workload on the oracle (all host
+    cores): the activation quantisation and the GEMM of a sample of token
+    rows against a sample of weight rows over the whole K (the rate, ops per
+    second, depends on neither count).  The weight rows are quantised off the
+    clock, as the method does offline."""
+    import oracle
+    hi = host_info()
+    threads = oracle.use_threads(hi["nproc"])
+    try:
+        mx = cfg.dtype == bq_synth.MXFP8
+        n_rows = 256 if cfg.dtype == bq_synth.INT8 else 128
+        w = bq_synth.weights(cfg.N, cfg.K, cfg.w_std, cfg.seed).numpy()[:n_rows]
+        if mx:
+            qw, sw = oracle.mx_quant(w.astype(np.float64))
+        else:
+            qw, sw = oracle.quant_weight(w, cfg.block_n, cfg.block_k, cfg.dtype)
+        del w
+        rows = max(2 * threads, 8)
+        xb = bq_synth.bf16_bits(bq_synth.activations(rows, cfg.K, cfg.seed, cfg.n_outliers,
+                                                     cfg.outlier_scale))
+
+        def step():
+            t0 = time.perf_counter()
+            if mx:
+                qa, sa = oracle.mx_quant(oracle.bf16_to_f64(xb))
+                oracle.mx_gemm(qa, sa, qw, sw)
+            else:
+                qa, sa = oracle.quant_act(xb, cfg.block_k, cfg.dtype)
+                oracle.gemm(qa, sa, qw, sw, cfg.block_n, cfg.block_k, cfg.dtype)
+            return time.perf_counter() - t0
+
+        reps, dt = _timed_reps(step, seconds_target)
+    finally:
+        oracle.use_threads(1)
+    ops = 2.0 * rows * n_rows * cfg.K
+    return {"value": reps * ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} x ({rows} of {cfg.M} token rows: quantisation + GEMM against "
+                      f"{n_rows} of the {cfg.N} weight rows, K = {cfg.K}); C oracle on "
+                      f"{threads} threads; {dt:.1f} s"}
+
+
+def cpu_baseline_moe(seconds_target=4.0):
+    """The MoE layer on the oracle, stage by stage, on a bounded sample: the
+    permutation of all T x top-k pairs, then for expert 0 and a sample of
+    its rows the w13 GEMM, silu * up with its requantisation, the w2 GEMM,
+    and the weighted combine of the sampled tokens.  Each stage's rate is
+    reported in its own unit; `value` is the layer's ops per second over the
+    two grouped GEMMs' sampled rows."""
+    import oracle
+    cfg = bq_synth.MOE
+    hi = host_info()
+    threads = oracle.use_threads(hi["nproc"])
+    try:
+        T, H, I, E, topk = cfg.T, cfg.H, cfg.I, cfg.E, cfg.topk
+        ids, tw = bq_synth.routing(T, E, topk, cfg.seed)
+        rows = max(2 * threads, 8)
+        # a sample of the expert's intermediate width: I2 gate rows, the
+        # matching up rows, and the w2 columns they feed
+        I2 = 256
+        w13 = bq_synth.weights(2 * I, H, cfg.w_std, cfg.seed).numpy()
+        w13 = np.concatenate([w13[:I2], w13[I:I + I2]])
+        q13, s13 = oracle.quant_weight_gate_up(w13, I2, 128, 128, cfg.dtype)
+        del w13
+        w2 = np.ascontiguousarray(bq_synth.weights(H, I, cfg.w_std, cfg.seed + 1).numpy()[:, :I2])
+        q2, s2 = oracle.quant_weight(w2, 128, 128, cfg.dtype)
+        del w2
+        I = I2
+        xb = bq_synth.bf16_bits(bq_synth.activations(rows, H, cfg.seed))
+        stages = {}
+
+        def timed(fn):
+            t0 = time.perf_counter()
+            out = fn()
+            return out, time.perf_counter() - t0
+
+        (_, _, _), t_perm = timed(lambda: oracle.moe_permute(ids, E))
+        stages["permute"] = {"value": T * topk / t_perm / 1e6, "unit": "M pairs/s"}
+        tot_gemm, tot_t = 0.0, 0.0
+        for _ in range(max(1, int(seconds_target / 2))):
+            (qa, sa), t_q = timed(lambda: oracle.quant_act(xb, 128, cfg.dtype))
+            y13, t_13 = timed(lambda: oracle.gemm(qa, sa, q13, s13, 128, 128, cfg.dtype, seam=I))
+            y13b = oracle.bf16_from_f64(y13)
+            h, t_s = timed(lambda: oracle.silu_mul(y13b, I))
+            (qh, sh), t_hq = timed(lambda: oracle.quant_act(h, 128, cfg.dtype))
+            y2, t_2 = timed(lambda: oracle.gemm(qh, sh, q2, s2, 128, 128, cfg.dtype))
+            y2b = oracle.bf16_from_f64(y2)
+            inv = np.arange(rows, dtype=np.int32)
+            _, t_c = timed(lambda: oracle.moe_combine(y2b, inv, np.full((rows // topk, topk),
+                                                                        0.5, np.float32)))
+            tot_gemm += 2.0 * rows * (2 * I) * H + 2.0 * rows * H * I
+            tot_t += t_q + t_13 + t_s + t_hq + t_2 + t_c
+        stages["w13_gemm"] = {"value": 2.0 * rows * 2 * I * H / t_13 / 1e12, "unit": "TOPS"}
+        stages["silu_requant"] = {"value": rows * I / (t_s + t_hq) / 1e6, "unit": "M elem/s"}
+        stages["w2_gemm"] = {"value": 2.0 * rows * H * I / t_2 / 1e12, "unit": "TOPS"}
+        stages["combine"] = {"value": rows * H / t_c / 1e6, "unit": "M elem/s"}
+    finally:
+        oracle.use_threads(1)
+    return {"value": tot_gemm / tot_t / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "stages": stages,
+            "sample": f"permute of all {T * topk} pairs; expert 0 with {rows} token rows and "
+                      f"{I} of its {cfg.I} intermediate columns through quant, w13, silu*up + "
+                      f"requant, w2 and combine; C oracle on {threads} threads; {tot_t:.1f} s"}
+
+
+def cpu_baseline_tiny():
+    """The tiny workload in full on the oracle, single-threaded: latency."""
+    import oracle
+    cfg = bq_synth.TINY
+    w = bq_synth.weights(cfg.N, cfg.K, cfg.w_std, cfg.seed).numpy()
+    qw, sw = oracle.quant_weight(w, cfg.block_n, cfg.block_k, cfg.dtype)
+    xb = bq_synth.bf16_bits(bq_synth.activations(cfg.M, cfg.K, cfg.seed, cfg.n_outliers,
+                                                 cfg.outlier_scale))
+
+    def step():
+        t0 = time.perf_counter()
+        qa, sa = oracle.quant_act(xb, cfg.block_k, cfg.dtype)
+        oracle.gemm(qa, sa, qw, sw, cfg.block_n, cfg.block_k, cfg.dtype)
+        return time.perf_counter() - t0
+
+    reps, dt = _timed_reps(step, 0.5)
+    return {"value": 1e6 * dt / reps, "unit": "us", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} whole tiny layers (quantisation + GEMM), single-threaded"}
 
 
 def run_reference(args):
@@ -653,10 +842,23 @@ def main():
                                                   bq_synth.MX_LINEAR, 3)
                 else:
                     subs[name] = bench_moe(args, dist, bq, peaks, stream)
+        if not args.no_sub:
+            torch.cuda.empty_cache()
+            subs["tiny"] = bench_tiny(args, dist, bq, stream)
     bq.check_device_status()
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         cpu = cpu_baseline()
+        # the other workloads' oracle baselines (bounded samples, all host cores)
+        big = {"prefill": bq_synth.PREFILL, "fp8": bq_synth.FP8_LINEAR,
+               "perchannel": bq_synth.PER_CHANNEL, "mxfp8": bq_synth.MX_LINEAR}
+        for name, sub in subs.items():
+            if name in big:
+                sub["cpu_baseline"] = cpu_baseline_linear(big[name])
+            elif name == "moe":
+                sub["cpu_baseline"] = cpu_baseline_moe()
+            elif name == "tiny":
+                sub["cpu_baseline"] = cpu_baseline_tiny()
     if dist.rank == 0:
         line = {"metric": METRIC, "value": head["value"], "unit": head["unit"],
                 "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,

@@ -2,7 +2,10 @@
 //
 //   SIMT     generic CUDA-core kernel: any shape, stride, block size.
 //   TCGEN05  TMA + tcgen05 kernel: block_n = block_k = 128, 16-byte strides.
-//   DECODE   swap-AB split-K weight-streaming tcgen05 kernel, M <= 128.
+//   DECODE   swap-AB split-K weight-streaming tcgen05 kernels, M <= 128: the
+//            cluster kernel of gemm_decode_cluster.cu (split-K reduced over
+//            distributed shared memory, no workspace) where it applies,
+//            else the workspace split-K kernel of gemm_decode.cu.
 //   GEMV     CUDA-core weight-streaming kernel, INT8, M <= 8 (forced only:
 //            measured on B200 it is no faster than DECODE at 1 token and
 //            slower at 8).
@@ -15,6 +18,7 @@
 #include "gemm_decode.h"
 #include "gemm_gemv.h"
 #include "gemm_tc.h"
+#include "gemm_decode_cluster.h"
 
 namespace bq {
 
@@ -69,6 +73,28 @@ static int run_decode(const GemmArgs& a, void* ws, size_t ws_bytes, bool pdl, cu
   return kRunOk;
 }
 
+// The cluster decode kernel.  Launched as a programmatic dependent of the
+// preceding kernel: it requests its weights before waiting for that kernel,
+// which therefore must not write them.
+static bool cluster_decode_args(const GemmArgs& a, DecClusterArgs* d) {
+  *d = DecClusterArgs{};
+  d->qa = a.qa; d->lda = a.lda; d->sa = a.sa;
+  d->qw = a.qw; d->ldw = a.ldw; d->sw = a.sw;
+  d->M = a.M; d->N = a.N; d->K = a.K; d->bn = a.bn; d->bk = a.bk;
+  d->dtype = a.dtype; d->bias = a.bias; d->out = a.out; d->ldo = a.ldo;
+  d->status = a.status; d->pdl = true;
+  return !a.offsets && a.sa_rows == a.M && gemm_decode_cluster_supported(*d, nullptr, 0);
+}
+
+static int run_cluster_decode(const DecClusterArgs& d, cudaStream_t st, char* why, size_t n) {
+  cudaError_t e = launch_gemm_decode_cluster(d, st);
+  if (e != cudaSuccess) {
+    snprintf(why, n, "decode GEMM launch: %s", cudaGetErrorString(e));
+    return kRunCuda;
+  }
+  return kRunOk;
+}
+
 static int run_gemv(const GemmArgs& a, bool pdl, cudaStream_t st, char* why, size_t n) {
   cudaError_t e = launch_gemm_gemv(a, pdl, st);
   if (e != cudaSuccess) {
@@ -81,14 +107,22 @@ static int run_gemv(const GemmArgs& a, bool pdl, cudaStream_t st, char* why, siz
 static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes, bool pdl,
                           cudaStream_t st, char* why, size_t why_len) {
   switch (path) {
-    case BQ_PATH_AUTO:
+    case BQ_PATH_AUTO: {
+      DecClusterArgs d;
+      if (a.M <= kDecodeMaxRows && cluster_decode_args(a, &d))
+        return run_cluster_decode(d, st, why, why_len);
       if (a.M <= kDecodeMaxRows && decode_supported(a, nullptr, 0))
         return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
       if (a.M > kDecodeMaxRows && tc_supported(a, nullptr, 0)) return run_tc(a, st, why, why_len);
       return run_simt(a, st, why, why_len);
-    case BQ_PATH_DECODE:
+    }
+    case BQ_PATH_DECODE: {
+      DecClusterArgs d;
+      if (a.M <= kDecodeMaxRows && cluster_decode_args(a, &d))
+        return run_cluster_decode(d, st, why, why_len);
       if (!decode_supported(a, why, why_len)) return kRunUnsupported;
       return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
+    }
     case BQ_PATH_GEMV:
       if (!gemv_supported(a, why, why_len)) return kRunUnsupported;
       return run_gemv(a, pdl, st, why, why_len);

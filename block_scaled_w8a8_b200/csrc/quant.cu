@@ -266,6 +266,9 @@ quant_weight_kernel(const float* __restrict__ w, int64_t N, int64_t K, int64_t l
     q[(n0 + r) * ldq + k0 + c] = one_code<DT>(w[(n0 + r) * ldw + k0 + c], sc);
   }
   if (threadIdx.x == 0) s[i * Kb + j] = sc;
+  // the decode kernels read weights before their dependency wait: make
+  // these codes visible GPU-wide before this CTA exits
+  __threadfence();
 }
 
 inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }

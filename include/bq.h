@@ -182,7 +182,10 @@ bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_
  * bias: bf16 [N] or NULL; out: bf16 [M, N] (row stride ldo >= N).
  * block_k <= 65536 keeps INT8 block partials exact in int32.
  * Kernels (BQ_PATH_AUTO): block_n = block_k = 128 with M <= 128 runs the
- *   split-K decode kernel; M > 128 runs the tcgen05 kernel, which promotes
+ *   split-K decode kernel (its K-splits reduced inside thread-block clusters;
+ *   split K ranges too long for its shared memory -- K above 65536, or above
+ *   32768 for M > 32 -- run the split-K kernel that reduces through the
+ *   workspace instead); M > 128 runs the tcgen05 kernel, which promotes
  *   each 128-wide K-block.  block_k >= K (one scale per token and per
  *   block_n rows of W: per-token / per-channel W8A8 with block_n = 1) also
  *   runs the tcgen05 kernel for M > 128, which then accumulates all of K in
@@ -190,6 +193,12 @@ bq_status bq_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int64_t block_
  *   The tensor-core kernels need 16-byte aligned operands with row strides
  *   that are multiples of 16 bytes; everything else runs the CUDA-core
  *   kernel.
+ * Stream overlap: the decode kernel starts as a programmatic dependent of
+ *   the kernel before it on the stream and requests its weight codes and
+ *   scales BEFORE waiting for that kernel to finish (activations, bias and
+ *   output are touched only after the wait).  The weights must therefore not
+ *   be written by the kernel immediately preceding this call on the stream
+ *   (libbq's own bq_quant_weight makes its writes visible before it exits).
  * workspace: device memory of at least bq_gemm_workspace_size bytes (may be
  *   NULL when that size is 0).  Its first 64 KiB hold arrival counters: they
  *   must be zero before the workspace is first used, and every completed
@@ -243,7 +252,9 @@ bq_status bq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int64_t bloc
  * i.e. apply_w8a8_block_int8_linear(input, weight, block_size, weight_scale,
  * input_scale=None, bias) of the block-wise INT8 page, section 4.
  * x: bf16 [M, K] (row stride ldx >= K); other arguments as bq_gemm.  The
- * workspace (bq_linear_workspace_size bytes) follows bq_gemm's rules. */
+ * workspace (bq_linear_workspace_size bytes) follows bq_gemm's rules.  The
+ * GEMM starts as a programmatic dependent of the quantiser, so its weight
+ * stream overlaps the quantisation (bq_gemm's stream-overlap rule applies). */
 bq_status bq_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void* qw,
                     int64_t ldw, const float* sw, int64_t N, int64_t block_n, int64_t block_k,
                     int dtype, const void* bias, void* out, int64_t ldo, void* workspace,

@@ -36,22 +36,44 @@ FP8 = 1
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bq_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "_bq_oracle.so")
+_LIB_OMP_PATH = os.path.join(_HERE, "_bq_oracle_omp.so")
 _lock = threading.Lock()
 _lib = None
+_lib_omp = None
+_use_omp = False
 
 # gcc flags: IEEE semantics, no fast-math, no FTZ.
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off"]
 
 
-def build(force: bool = False) -> str:
-    """Compile bq_oracle.c into _bq_oracle.so next to it (if stale)."""
-    stale = (not os.path.exists(_LIB_PATH)) or (
-        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+def _build_one(path: str, extra, force: bool) -> str:
+    stale = (not os.path.exists(path)) or os.path.getmtime(path) < os.path.getmtime(_SRC)
     if force or stale:
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+        tmp = path + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, *extra, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, path)
+    return path
+
+
+def build(force: bool = False) -> str:
+    """Compile bq_oracle.c into _bq_oracle.so next to it (if stale), and the
+    same source with -fopenmp into _bq_oracle_omp.so: its row loops then run
+    on several threads (same arithmetic per element; used only to time the
+    CPU baseline on all host cores)."""
+    _build_one(_LIB_OMP_PATH, ["-fopenmp"], force)
+    return _build_one(_LIB_PATH, [], force)
+
+
+def use_threads(n: int) -> int:
+    """Run the oracle's row loops on n threads (the OpenMP build) when n > 1,
+    or on one thread (the plain build) when n <= 1.  Returns the thread count
+    now in use.  Results are identical either way: every output element is
+    computed by the same code, only rows are split over threads."""
+    global _use_omp
+    with _lock:
+        _use_omp = n > 1
+    lib = _load()
+    return int(lib.bq_ref_threads(n if n > 1 else 1))
 
 
 def configure(lib):
@@ -85,16 +107,19 @@ def configure(lib):
     lib.bq_ref_mx_quant.restype = None
     lib.bq_ref_mx_gemm.argtypes = [P, L, P, P, L, P, L, L, L, P, P]
     lib.bq_ref_mx_gemm.restype = None
+    lib.bq_ref_threads.argtypes = [I]
+    lib.bq_ref_threads.restype = I
     return lib
 
 
 def _load():
-    global _lib
+    global _lib, _lib_omp
     with _lock:
-        if _lib is None:
+        if _lib is None or _lib_omp is None:
             build()
             _lib = configure(ctypes.CDLL(_LIB_PATH))
-    return _lib
+            _lib_omp = configure(ctypes.CDLL(_LIB_OMP_PATH))
+        return _lib_omp if _use_omp else _lib
 
 
 def _ptr(a: np.ndarray | None):

@@ -182,17 +182,23 @@ static double code_value(uint8_t c, int dtype) {
 void bq_ref_quant_act(const uint16_t* x, long M, long K, long ldx, long group_k,
                       int dtype, uint8_t* q, long ldq, float* s) {
     long Kb = (K + group_k - 1) / group_k;
-    float* buf = (float*)malloc(sizeof(float) * (size_t)(group_k > 0 ? group_k : 1));
-    for (long m = 0; m < M; m++) {
-        for (long g = 0; g < Kb; g++) {
-            long k0 = g * group_k;
-            long L = (k0 + group_k <= K) ? group_k : K - k0;
-            for (long i = 0; i < L; i++)
-                buf[i] = (float)bq_ref_bf16_to_double(x[m * ldx + k0 + i]);
-            s[m * Kb + g] = quant_group(buf, L, dtype, q + m * ldq + k0);
+    /* rows are independent: the OpenMP build (baseline timing only) splits
+     * them over threads; without -fopenmp the pragmas are ignored */
+#pragma omp parallel
+    {
+        float* buf = (float*)malloc(sizeof(float) * (size_t)(group_k > 0 ? group_k : 1));
+#pragma omp for schedule(static)
+        for (long m = 0; m < M; m++) {
+            for (long g = 0; g < Kb; g++) {
+                long k0 = g * group_k;
+                long L = (k0 + group_k <= K) ? group_k : K - k0;
+                for (long i = 0; i < L; i++)
+                    buf[i] = (float)bq_ref_bf16_to_double(x[m * ldx + k0 + i]);
+                s[m * Kb + g] = quant_group(buf, L, dtype, q + m * ldq + k0);
+            }
         }
+        free(buf);
     }
-    free(buf);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -272,6 +278,7 @@ double bq_ref_gemm_entry(const uint8_t* qa, long lda, const float* sa, const uin
 void bq_ref_gemm(const uint8_t* qa, long lda, const float* sa, const uint8_t* qw,
                  long ldw, const float* sw, long M, long N, long K, long bn, long bk,
                  long seam, int dtype, const uint16_t* bias, double* out) {
+#pragma omp parallel for schedule(static)
     for (long m = 0; m < M; m++)
         for (long n = 0; n < N; n++)
             out[m * N + n] = bq_ref_gemm_entry(qa, lda, sa, qw, ldw, sw, N, K, bn, bk, seam,
@@ -328,6 +335,7 @@ int bq_ref_moe_permute(const int32_t* ids, long T, long topk, long E, int32_t* o
  * ("gate + up fused", [BWI8] §5; SiLU is the reading for a gate/up pair).
  * silu(g) = g / (1 + exp(-g)), in fp64. */
 void bq_ref_silu_mul(const uint16_t* y, long R, long I, long ldy, uint16_t* h) {
+#pragma omp parallel for schedule(static)
     for (long r = 0; r < R; r++) {
         for (long i = 0; i < I; i++) {
             double g = bq_ref_bf16_to_double(y[r * ldy + i]);
@@ -341,6 +349,7 @@ void bq_ref_silu_mul(const uint16_t* y, long R, long I, long ldy, uint16_t* h) {
 /* out[t, n] = bf16( sum_j w[t, j] * y[inv_perm[t*topk + j], n] ), fp64. */
 void bq_ref_moe_combine(const uint16_t* y, long ldy, const int32_t* inv_perm,
                         const float* w, long T, long topk, long H, uint16_t* out) {
+#pragma omp parallel for schedule(static)
     for (long t = 0; t < T; t++) {
         for (long n = 0; n < H; n++) {
             double acc = 0.0;
@@ -413,6 +422,7 @@ void bq_ref_mx_gemm(const uint8_t* qa, long lda, const uint8_t* sa, const uint8_
                     long ldw, const uint8_t* sw, long M, long N, long K,
                     const uint16_t* bias, double* out) {
     long G = (K + BQ_REF_MX_GROUP - 1) / BQ_REF_MX_GROUP;
+#pragma omp parallel for schedule(static)
     for (long m = 0; m < M; m++)
         for (long n = 0; n < N; n++) {
             double acc = 0.0;
@@ -429,3 +439,19 @@ void bq_ref_mx_gemm(const uint8_t* qa, long lda, const uint8_t* sa, const uint8_
             out[m * N + n] = acc;
         }
 }
+
+/* Threads used by the row loops above: the OpenMP build (compiled with
+ * -fopenmp, for the CPU baseline timing) sets and reports them; the plain
+ * build always runs one thread. */
+#ifdef _OPENMP
+#include <omp.h>
+int bq_ref_threads(int n) {
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+}
+#else
+int bq_ref_threads(int n) {
+    (void)n;
+    return 1;
+}
+#endif

@@ -240,17 +240,21 @@ def test_linear_decode_path_with_dependent_launch(M):
     assert all(torch.equal(outs[0], o) for o in outs[1:])
 
 
-# Shapes on which bq_linear runs the fused decode kernel (the kernel quantises
-# its own K slice of x): M <= 32, at least 16 weight tiles, x 16-byte aligned
-# with a row stride that is a multiple of 8.  Partial K-blocks, K not a
-# multiple of 8 (row stride padded), ragged N and bias are all covered.
-FUSED_SHAPES = [(1, 2048, 4096, 4096), (5, 4096, 1000, 1000), (16, 2048, 1004, 1008),
-                (17, 3000, 4096, 4096), (32, 4096, 8192, 8192), (3, 2100, 300, 304)]
+# bq_linear with M <= 128: the activation quantiser, then the cluster decode
+# GEMM (split-K reduced over distributed shared memory) as a programmatic
+# dependent of it.  The shapes cover clusters of 1 to 8 K-splits (N = 128 up
+# to 4096, 3000 ragged), every token tile (16, 32, 64, 128), token counts
+# that are not multiples of 16, partial K-blocks, x rows not 16-byte aligned
+# (K = 1000), padded row strides and bias.
+LINEAR_DECODE_SHAPES = [(1, 2048, 4096, 4096), (5, 4096, 1000, 1000), (16, 2048, 1004, 1008),
+                (17, 3000, 4096, 4096), (32, 4096, 8192, 8192), (3, 2100, 300, 304),
+                (33, 4096, 4096, 4096), (64, 4096, 4096, 4096), (64, 640, 1008, 1008),
+                (100, 1024, 2048, 2056), (128, 4096, 1024, 1024), (1, 128, 128, 128)]
 
 
 @pytest.mark.parametrize("dtype", [INT8, FP8])
-@pytest.mark.parametrize("M,N,K,ldx", FUSED_SHAPES)
-def test_linear_fused_decode_vs_oracle(M, N, K, ldx, dtype):
+@pytest.mark.parametrize("M,N,K,ldx", LINEAR_DECODE_SHAPES)
+def test_linear_decode_vs_oracle(M, N, K, ldx, dtype):
     xb = act_bits(M, K, 90 + M, 7, 25.0)
     w = bq_synth.weights(N, K, 0.02, 91 + M).numpy()
     qw, sw = oracle.quant_weight(w, 128, 128, dtype)
@@ -265,19 +269,20 @@ def test_linear_fused_decode_vs_oracle(M, N, K, ldx, dtype):
     bq.check_device_status()
     qa, sa = oracle.quant_act(xb, 128, dtype)
     ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bias)
-    assert_gemm_close(outs[0], ref, f"fused linear M={M} N={N} K={K}")
+    assert_gemm_close(outs[0], ref, f"linear decode M={M} N={N} K={K}")
     assert torch.equal(outs[0], outs[1])
 
 
 @pytest.mark.parametrize("dtype", [INT8, FP8])
-@pytest.mark.parametrize("M", [1, 7, 32])
-def test_linear_fused_codes_exact_through_identity_weight(M, dtype):
+@pytest.mark.parametrize("M", [1, 7, 32, 33, 64, 128])
+def test_linear_decode_codes_exact_through_identity_weight(M, dtype):
     """With W = identity (code of 1.0, block scale 1) each output is
     bf16(fl32(q[t, n] * sa[t, n // 128])): one product, rounded to fp32 by the
     kernel's promotion FMA, then to bf16.  Neighbouring INT8 codes (and e4m3
     codes) differ by at least 1/127 (1/8) relatively, more than a bf16 ulp,
-    so any wrong code or misplaced swizzle slot of the fused quantiser shows
-    as an exact mismatch against the oracle's codes."""
+    so any wrong code, misplaced activation tile, or partial summed into the
+    wrong row by the cluster reduction shows as an exact mismatch against the
+    oracle's codes."""
     N = K = 2048
     xb = act_bits(M, K, 300 + M, 11, 40.0)
     one = 1 if dtype == INT8 else int(oracle.e4m3_encode(np.array([1.0]))[0])
@@ -720,13 +725,15 @@ def test_shared_workspace_survives_every_entry_point():
     w = bq_synth.weights(N, K, 0.02, 721).numpy()
     qw, sfw = bq.mx_quant_weight(torch.from_numpy(w).cuda())
     x = dev_bf16(xb)
-    need = max(bq.mx_linear_workspace_size(M, K), bq.gemm_workspace_size(1, 640, 1008),
-               bq.linear_workspace_size(33, 1000, 2048))
+    need = max(bq.mx_linear_workspace_size(M, K), bq.gemm_workspace_size(1, 640, 66560),
+               bq.linear_workspace_size(33, 256, 33024))
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     bq.mx_linear(x, qw, sfw, ws=ws)
     torch.cuda.synchronize()
     assert int(ws[:65536].count_nonzero()) == 0, "bq_mx_linear wrote into the counter region"
-    for (Md, Nd, Kd), seed in (((1, 640, 1008), 722), ((33, 1000, 2048), 723)):
+    # split K ranges too long for the cluster kernel's shared memory: these
+    # run the split-K kernel that reduces through the workspace
+    for (Md, Nd, Kd), seed in (((1, 640, 66560), 722), ((33, 256, 33024), 723)):
         xd, qa, sa, qwd, swd, _ = make_problem(Md, Nd, Kd, 128, 128, INT8, seed)
         ref = oracle.gemm(qa, sa, qwd, swd, 128, 128, INT8)
         assert bq.gemm_workspace_size(Md, Nd, Kd) > 0, "shape must use the workspace"

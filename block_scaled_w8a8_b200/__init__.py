@@ -22,8 +22,7 @@ import torch
 INT8 = 0
 FP8_E4M3 = 1
 
-PATH_AUTO, PATH_SIMT, PATH_TCGEN05, PATH_DECODE, PATH_TCGEN05_1CTA, PATH_TCGEN05_2CTA, \
-    PATH_GEMV = 0, 1, 2, 3, 4, 5, 6
+PATH_AUTO, PATH_SIMT, PATH_TCGEN05, PATH_DECODE, PATH_TCGEN05_1CTA = 0, 1, 2, 3, 4
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT = range(7)
@@ -50,6 +49,9 @@ DECLS = {
     "bq_gemm_workspace_size": (_INT, [_I64, _I64, _I64, _I64, _I64, _INT, _SZP]),
     "bq_gemm": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _I64, _I64, _INT, _P, _P,
                        _I64, _P, _SZ, _P]),
+    "bq_gemm_partial": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _I64, _I64, _INT,
+                               _P, _I64, _P, _SZ, _P]),
+    "bq_finish_bf16": (_INT, [_P, _I64, _I64, _I64, _P, _P, _I64, _P]),
     "bq_gemm_decode_noalloc": (_INT, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _I64, _I64,
                                       _INT, _P, _P, _I64, _P]),
     "bq_linear_workspace_size": (_INT, [_I64, _I64, _I64, _I64, _I64, _INT, _SZP]),
@@ -234,6 +236,33 @@ def gemm(qa, sa, qw, sw, block_n=128, block_k=128, dtype=INT8, bias=None, out=No
                          _cuda(sw, "sw"), M, N, K, block_n, block_k, dtype,
                          _opt(bias, "bias"), _cuda(out, "out"), _ld(out), _opt(ws, "ws"),
                          0 if ws is None else ws.numel(), _P(_stream(qa.device))))
+    return out
+
+
+def gemm_partial(qa, sa, qw, sw, block_n=128, block_k=128, dtype=INT8, out=None, ws=None):
+    """Unrounded fp32 sum over the K-blocks of qa/qw (no bias): the per-GPU
+    part of a K-sharded linear layer, finished by finish_bf16."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float32, device=qa.device)
+    nbytes = gemm_workspace_size(M, N, K, block_n, block_k, dtype)
+    if ws is None:
+        ws = workspace(nbytes, qa.device)
+    _check(lib().bq_gemm_partial(_cuda(qa, "qa"), _ld(qa), _cuda(sa, "sa"), _cuda(qw, "qw"),
+                                 _ld(qw), _cuda(sw, "sw"), M, N, K, block_n, block_k, dtype,
+                                 _cuda(out, "out"), _ld(out), _opt(ws, "ws"),
+                                 0 if ws is None else ws.numel(), _P(_stream(qa.device))))
+    return out
+
+
+def finish_bf16(part, bias=None, out=None):
+    """bf16(part + bias), one rounding."""
+    M, N = part.shape
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=part.device)
+    _check(lib().bq_finish_bf16(_cuda(part, "part"), _ld(part), M, N, _opt(bias, "bias"),
+                                _cuda(out, "out"), _ld(out), _P(_stream(part.device))))
     return out
 
 

@@ -100,7 +100,7 @@ const char* bq_status_string(int s) {
 const char* bq_last_error_message(void) { return g_msg; }
 
 bq_status bq_set_path(int path) {
-  BQ_CHECK_ARG(path >= BQ_PATH_AUTO && path <= BQ_PATH_GEMV, "unknown path %d", path);
+  BQ_CHECK_ARG(path >= BQ_PATH_AUTO && path <= BQ_PATH_TCGEN05_1CTA, "unknown path %d", path);
   g_path = path;
   return ok();
 }
@@ -253,6 +253,54 @@ static bq_status gemm_impl(const void* qa, int64_t lda, const float* sa, const v
   if (rc == bq::kRunUnsupported) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
   if (rc == bq::kRunAlignment) return fail(BQ_ERR_ALIGNMENT, "%s", why);
   return fail(BQ_ERR_CUDA, "%s", why);
+}
+
+bq_status bq_gemm_partial(const void* qa, int64_t lda, const float* sa, const void* qw,
+                          int64_t ldw, const float* sw, int64_t M, int64_t N, int64_t K,
+                          int64_t block_n, int64_t block_k, int dtype, float* out, int64_t ldo,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  bq_status st = check_gemm_shape(M, N, K, block_n, block_k, dtype);
+  if (st != BQ_OK) return st;
+  BQ_CHECK_ARG(lda >= K && ldw >= K && ldo >= N, "leading dimensions too small");
+  if (M == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(out, "out must not be NULL");
+  if (K == 0) {
+    for (int64_t m = 0; m < M; ++m)
+      BQ_CHECK_CUDA(cudaMemsetAsync(out + m * ldo, 0, (size_t)N * sizeof(float), as_stream(stream)),
+                    "zero partial");
+    return ok();
+  }
+  BQ_CHECK_ARG(qa && sa && qw && sw, "qa, sa, qw and sw must not be NULL");
+  unsigned* w = nullptr;
+  st = status_word(&w);
+  if (st != BQ_OK) return st;
+  bq::GemmArgs a{};
+  a.qa = qa; a.lda = lda; a.sa = sa; a.sa_rows = M;
+  a.qw = qw; a.ldw = ldw; a.sw = sw;
+  a.M = M; a.N = N; a.K = K; a.bn = block_n; a.bk = block_k; a.seam = 0;
+  a.Nbs = cdiv(N, block_n);
+  a.dtype = dtype; a.bias = nullptr; a.out = nullptr; a.ldo = ldo;
+  a.offsets = nullptr; a.E = 1; a.w_expert_stride = 0; a.sw_expert_stride = 0;
+  a.status = w;
+  a.out_f32 = out;
+  char why[256] = "";
+  const int rc = bq::run_gemm(a, g_path, workspace, workspace_bytes, as_stream(stream), why,
+                              sizeof(why));
+  if (rc == bq::kRunOk) return ok();
+  if (rc == bq::kRunUnsupported) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
+  if (rc == bq::kRunAlignment) return fail(BQ_ERR_ALIGNMENT, "%s", why);
+  return fail(BQ_ERR_CUDA, "%s", why);
+}
+
+bq_status bq_finish_bf16(const float* part, int64_t ldp, int64_t M, int64_t N, const void* bias,
+                         void* out, int64_t ldo, void* stream) {
+  BQ_CHECK_ARG(M >= 0 && N >= 0, "M and N must be >= 0");
+  BQ_CHECK_ARG(ldp >= N && ldo >= N, "leading dimensions too small");
+  if (M == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(part && out, "part and out must not be NULL");
+  BQ_CHECK_CUDA(bq::launch_finish_bf16(part, ldp, M, N, bias, out, ldo, as_stream(stream)),
+                "finish_bf16 launch");
+  return ok();
 }
 
 bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, int64_t ldw,

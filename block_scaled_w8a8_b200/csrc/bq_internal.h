@@ -44,6 +44,9 @@ struct GemmArgs {
   // is set, out is unused and the kernel writes codes [M, seam] (row stride
   // ldq) and scales [seam / 128][sa_rows]
   void* q_out; int64_t ldq; float* s_out;
+  // fp32 partial output (bq_gemm_partial): when set, out and bias are unused
+  // and the kernel stores sum_kb P_kb * sa * sw unrounded to out_f32 [M, ldo]
+  float* out_f32;
 };
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
@@ -55,6 +58,10 @@ cudaError_t launch_moe_permute(const int32_t* ids, int64_t T, int64_t topk, int6
 cudaError_t launch_moe_combine(const void* y, int64_t ldy, const int32_t* inv_perm,
                                const float* w, int64_t T, int64_t topk, int64_t H, void* out,
                                int64_t ldo, cudaStream_t st);
+
+// out = bf16(part + bias): the single rounding after a K-sharded sum.
+cudaError_t launch_finish_bf16(const float* part, int64_t ldp, int64_t M, int64_t N,
+                               const void* bias, void* out, int64_t ldo, cudaStream_t st);
 
 // Bounded-wait self-test.
 cudaError_t launch_selftest_wait(int64_t spin_limit, unsigned* status, cudaStream_t st);

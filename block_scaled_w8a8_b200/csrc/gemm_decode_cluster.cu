@@ -67,6 +67,7 @@ struct DecParams {
   int S;                                      // CTAs (K-splits) per tile
   const uint16_t* bias;
   uint16_t* out; int64_t ldo;
+  float* out_f32;                             // unrounded fp32 output (no bias) or null
   unsigned* status;
 };
 
@@ -453,8 +454,14 @@ gemm_decode_cluster_kernel(const __grid_constant__ CUtensorMap tmW,
             *reinterpret_cast<const float4*>(slots + (src * R + rr) * L::kNtp + 4 * tq);
         sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
       }
-      const float bv = p.bias ? bf16_bits_to_float(p.bias[n]) : 0.0f;
       const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+      if (p.out_f32) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * tq + e < M) p.out_f32[(int64_t)(4 * tq + e) * p.ldo + n] = vals[e];
+        continue;
+      }
+      const float bv = p.bias ? bf16_bits_to_float(p.bias[n]) : 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if (4 * tq + e < M)
@@ -520,6 +527,7 @@ cudaError_t launch_one(const DecClusterArgs& a, const DecClusterPlan& plan, cuda
   p.S = plan.S;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.out = static_cast<uint16_t*>(a.out); p.ldo = a.ldo;
+  p.out_f32 = a.out_f32;
   p.status = a.status;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(plan.tiles * p.S), 1, 1);

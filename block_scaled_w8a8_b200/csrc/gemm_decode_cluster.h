@@ -17,6 +17,7 @@ struct DecClusterArgs {
   int dtype;
   const void* bias;                    // bf16 [N] or nullptr
   void* out; int64_t ldo;              // bf16 [M, ldo]
+  float* out_f32;                      // or: unrounded fp32 [M, ldo], no bias
   unsigned* status;
   bool pdl;                            // programmatic dependent launch
 };

@@ -6,9 +6,6 @@
 //            cluster kernel of gemm_decode_cluster.cu (split-K reduced over
 //            distributed shared memory, no workspace) where it applies,
 //            else the workspace split-K kernel of gemm_decode.cu.
-//   GEMV     CUDA-core weight-streaming kernel, INT8, M <= 8 (forced only:
-//            measured on B200 it is no faster than DECODE at 1 token and
-//            slower at 8).
 // AUTO: M <= 128 -> DECODE, larger M -> TCGEN05, when they apply; otherwise
 // the generic CUDA-core kernel.
 #include <cstdio>
@@ -16,7 +13,6 @@
 #include "bq.h"
 #include "gemm_paths.h"
 #include "gemm_decode.h"
-#include "gemm_gemv.h"
 #include "gemm_tc.h"
 #include "gemm_decode_cluster.h"
 
@@ -42,15 +38,8 @@ static int run_simt(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
   return kRunOk;
 }
 
-// kind: 0 = default tcgen05 kernel, 1 = 1-CTA, 2 = CTA pair.  Measured on
-// B200 the CTA-pair kernel is slower than the 1-CTA kernel for every workload
-// here (its epilogue drains TMEM more slowly), so it runs only when forced.
-// Tile width of the CTA-pair kernel (128 or 256; 256 measured faster).
-static int g_pair_tile_n = 256;
-
-static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n, int kind = 0) {
-  const bool pair = kind == 2;
-  cudaError_t e = pair ? launch_gemm_tc_pair(a, g_pair_tile_n, st) : launch_gemm_tc(a, st);
+static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
+  cudaError_t e = launch_gemm_tc(a, st);
   if (e != cudaSuccess) {
     snprintf(why, n, "tcgen05 GEMM launch: %s", cudaGetErrorString(e));
     return kRunCuda;
@@ -82,6 +71,7 @@ static bool cluster_decode_args(const GemmArgs& a, DecClusterArgs* d) {
   d->qw = a.qw; d->ldw = a.ldw; d->sw = a.sw;
   d->M = a.M; d->N = a.N; d->K = a.K; d->bn = a.bn; d->bk = a.bk;
   d->dtype = a.dtype; d->bias = a.bias; d->out = a.out; d->ldo = a.ldo;
+  d->out_f32 = a.out_f32;
   d->status = a.status; d->pdl = true;
   return !a.offsets && a.sa_rows == a.M && gemm_decode_cluster_supported(*d, nullptr, 0);
 }
@@ -95,15 +85,6 @@ static int run_cluster_decode(const DecClusterArgs& d, cudaStream_t st, char* wh
   return kRunOk;
 }
 
-static int run_gemv(const GemmArgs& a, bool pdl, cudaStream_t st, char* why, size_t n) {
-  cudaError_t e = launch_gemm_gemv(a, pdl, st);
-  if (e != cudaSuccess) {
-    snprintf(why, n, "CUDA-core decode launch: %s", cudaGetErrorString(e));
-    return kRunCuda;
-  }
-  return kRunOk;
-}
-
 static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes, bool pdl,
                           cudaStream_t st, char* why, size_t why_len) {
   switch (path) {
@@ -111,7 +92,7 @@ static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes
       DecClusterArgs d;
       if (a.M <= kDecodeMaxRows && cluster_decode_args(a, &d))
         return run_cluster_decode(d, st, why, why_len);
-      if (a.M <= kDecodeMaxRows && decode_supported(a, nullptr, 0))
+      if (a.M <= kDecodeMaxRows && !a.out_f32 && decode_supported(a, nullptr, 0))
         return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
       if (a.M > kDecodeMaxRows && tc_supported(a, nullptr, 0)) return run_tc(a, st, why, why_len);
       return run_simt(a, st, why, why_len);
@@ -120,19 +101,19 @@ static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes
       DecClusterArgs d;
       if (a.M <= kDecodeMaxRows && cluster_decode_args(a, &d))
         return run_cluster_decode(d, st, why, why_len);
+      if (a.out_f32) {
+        snprintf(why, why_len, "decode path: fp32 partial output needs the cluster kernel");
+        return kRunUnsupported;
+      }
       if (!decode_supported(a, why, why_len)) return kRunUnsupported;
       return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
     }
-    case BQ_PATH_GEMV:
-      if (!gemv_supported(a, why, why_len)) return kRunUnsupported;
-      return run_gemv(a, pdl, st, why, why_len);
     case BQ_PATH_SIMT:
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
     case BQ_PATH_TCGEN05_1CTA:
-    case BQ_PATH_TCGEN05_2CTA:
       if (!tc_supported(a, why, why_len)) return kRunUnsupported;
-      return run_tc(a, st, why, why_len, path == BQ_PATH_TCGEN05 ? 0 : path - 3);
+      return run_tc(a, st, why, why_len);
     default:
       snprintf(why, why_len, "kernel path %d is not available in this build", path);
       return kRunUnsupported;
@@ -161,9 +142,8 @@ int run_grouped_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cud
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
     case BQ_PATH_TCGEN05_1CTA:
-    case BQ_PATH_TCGEN05_2CTA:
       if (!tc_supported(a, why, why_len)) return kRunUnsupported;
-      return run_tc(a, st, why, why_len, path == BQ_PATH_TCGEN05 ? 0 : path - 3);
+      return run_tc(a, st, why, why_len);
     default:
       snprintf(why, why_len, "kernel path %d is not available for grouped GEMM", path);
       return kRunUnsupported;

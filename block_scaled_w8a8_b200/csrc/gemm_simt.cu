@@ -137,6 +137,10 @@ gemm_simt_kernel(GemmArgs a) {
       const int64_t gn = nt + tx + 16 * j;
       if (gn >= a.N) continue;
       float v = acc[i][j];
+      if (a.out_f32) {
+        a.out_f32[(row0 + gm) * a.ldo + gn] = v;
+        continue;
+      }
       if (bias) v += bf16_bits_to_float(bias[gn]);
       out[gm * a.ldo + gn] = float_to_bf16_bits(v);
     }

@@ -459,7 +459,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ++tcount;
         continue;
       }
-      if (row_ok && n0 < p.N) {
+      if (row_ok && n0 < p.N && p.out_f32) {
+        float* frow = p.out_f32 + m * p.ldo + n0;
+        if (n0 + CW <= p.N && ((reinterpret_cast<uintptr_t>(frow) & 15) == 0)) {
+#pragma unroll
+          for (int j = 0; j < CW; j += 4)
+            *reinterpret_cast<float4*>(frow + j) =
+                make_float4(accf[j], accf[j + 1], accf[j + 2], accf[j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (n0 + j < p.N) frow[j] = accf[j];
+        }
+      } else if (row_ok && n0 < p.N) {
         uint16_t* orow = p.out + m * p.ldo + n0;
         const bool full_n = n0 + CW <= p.N;
         const bool vec = full_n && ((reinterpret_cast<uintptr_t>(orow) & 15) == 0);
@@ -539,6 +551,7 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   p.nblk = SILU ? (int)(a.seam / 128) : (int)((a.N + BN - 1) / BN);
   p.status = a.status;
   p.q_out = static_cast<uint8_t*>(a.q_out); p.ldq = a.ldq; p.s_out = a.s_out;
+  p.out_f32 = a.out_f32;
   const int64_t mblk_bound = (a.M + BM - 1) / BM + (a.offsets ? a.E : 0);
   const int64_t tiles_bound = mblk_bound * p.nblk;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles_bound, sm_count()));

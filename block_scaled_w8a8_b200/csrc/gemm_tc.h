@@ -17,8 +17,5 @@ bool tc_silu_supported(const GemmArgs& a, char* why, size_t n);
 cudaError_t launch_gemm_tc_silu(const GemmArgs& a, cudaStream_t st);
 // Single-CTA kernel: 128 x 256 tiles (128 x 128 for N <= 128).
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
-// CTA-pair kernel (cta_group::2): 256 x tile_n tiles (tile_n = 128 or 256);
-// same requirements.
-cudaError_t launch_gemm_tc_pair(const GemmArgs& a, int tile_n, cudaStream_t st);
 
 }  // namespace bq

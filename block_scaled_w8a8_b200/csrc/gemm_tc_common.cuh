@@ -33,6 +33,7 @@ struct TcParams {
   // fused SiLU * up + requantisation (gate/up weight, seam = I): codes of h
   // [rows, I] (row stride ldq) and scales [I / 128][sa_rows] instead of out
   uint8_t* q_out; int64_t ldq; float* s_out;
+  float* out_f32;                               // unrounded fp32 output (no bias) or null
 };
 
 // Weight-scale row of output column n (block_n = 128).  A fused gate+up

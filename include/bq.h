@@ -87,10 +87,7 @@ typedef enum bq_path {
     BQ_PATH_SIMT = 1,     /* generic CUDA-core kernel: any shape/stride */
     BQ_PATH_TCGEN05 = 2,  /* TMA + tcgen05 tensor-core kernel (large M) */
     BQ_PATH_DECODE = 3,   /* split-K weight-streaming kernel (small M) */
-    BQ_PATH_TCGEN05_1CTA = 4,  /* force the 1-CTA tcgen05 kernel (128x256 tiles) */
-    BQ_PATH_TCGEN05_2CTA = 5,  /* force the CTA-pair 256x256-tile kernel */
-    BQ_PATH_GEMV = 6      /* CUDA-core weight-streaming kernel, INT8, M <= 8
-                             (forced only) */
+    BQ_PATH_TCGEN05_1CTA = 4   /* force the tcgen05 kernel (128x256 tiles) */
 } bq_path;
 
 /* ---- library information and errors ---------------------------------- */
@@ -217,6 +214,29 @@ bq_status bq_gemm(const void* qa, int64_t lda, const float* sa, const void* qw, 
                   const float* sw, int64_t M, int64_t N, int64_t K, int64_t block_n,
                   int64_t block_k, int dtype, const void* bias, void* out, int64_t ldo,
                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same contraction as bq_gemm without the last step: out (fp32 [M, N],
+ * row stride ldo >= N) = sum_kb P_kb[m,n] * sa[kb*M + m] * sw[(n/block_n)*Kb + kb],
+ * unrounded and without bias.  This is the per-GPU part of a linear layer
+ * whose K dimension is split over GPUs (row-parallel tensor parallelism,
+ * block-wise INT8 page, section 3: each GPU's input_size_per_partition is a
+ * multiple of block_k, so its activation groups and weight blocks are whole):
+ * the partials of all shards are summed in fp32 (an all-reduce or a
+ * reduce-scatter), then bq_finish_bf16 adds the bias and rounds once, as the
+ * unsharded layer does.  Arguments and kernels as bq_gemm; the decode path
+ * needs the cluster kernel (the fallback is the CUDA-core kernel).  K = 0
+ * writes zeros. */
+bq_status bq_gemm_partial(const void* qa, int64_t lda, const float* sa, const void* qw,
+                          int64_t ldw, const float* sw, int64_t M, int64_t N, int64_t K,
+                          int64_t block_n, int64_t block_k, int dtype, float* out, int64_t ldo,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* out[m, n] = bf16(part[m, n] + bias[n]) (one round-to-nearest-even; bias
+ * bf16 [N] or NULL): the single rounding that ends a K-sharded linear layer
+ * after its fp32 partials were summed (see bq_gemm_partial).  part: fp32
+ * [M, N] (row stride ldp >= N); out: bf16 [M, N] (row stride ldo >= N). */
+bq_status bq_finish_bf16(const float* part, int64_t ldp, int64_t M, int64_t N, const void* bias,
+                         void* out, int64_t ldo, void* stream);
 
 /* bq_gemm restricted to the split-K decode kernel, with NO workspace argument
  * and no device allocation: for callers that cannot allocate device memory

@@ -141,7 +141,7 @@ TC_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
+@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA])
 @pytest.mark.parametrize("dtype", [INT8, FP8])
 @pytest.mark.parametrize("M,N,K", TC_SHAPES)
 def test_gemm_tcgen05_vs_oracle(path, dtype, M, N, K):
@@ -194,33 +194,6 @@ def test_gemm_decode_vs_oracle(dtype, M, N, K):
     ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bb)
     assert_gemm_close(out1, ref, f"decode dtype={dtype} {M}x{N}x{K}")
     assert torch.equal(out1, out2), "split-K reduction is not deterministic"
-
-
-GEMV_SHAPES = [(1, 640, 1008), (2, 4096, 4096), (8, 4096, 4096), (5, 1000, 4112),
-               (8, 384, 8192), (3, 130, 256), (7, 256, 16), (4, 200, 6144)]
-
-
-@pytest.mark.parametrize("M,N,K", GEMV_SHAPES)
-def test_gemm_gemv_vs_oracle(M, N, K):
-    _, qa, sa, qw, sw, bb = make_problem(M, N, K, 128, 128, INT8, 700 + M, bias=(M % 2 == 0))
-    bq.set_path(bq.PATH_GEMV)
-    out = bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, INT8,
-                  bias=None if bb is None else dev_bf16(bb))
-    torch.cuda.synchronize()
-    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, INT8, bias_bf16=bb)
-    assert_gemm_close(out, ref, f"gemv {M}x{N}x{K}")
-
-
-def test_gemm_gemv_rejects_fp8_and_many_tokens():
-    bq.set_path(bq.PATH_GEMV)
-    _, qa, sa, qw, sw, _ = make_problem(9, 256, 256, 128, 128, INT8, 1)
-    with pytest.raises(bq.BqError) as ei:
-        bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, INT8)
-    assert ei.value.status == bq.ERR_UNSUPPORTED
-    _, qa, sa, qw, sw, _ = make_problem(4, 256, 256, 128, 128, FP8, 2)
-    with pytest.raises(bq.BqError) as ei:
-        bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, FP8)
-    assert ei.value.status == bq.ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("M", [1, 8, 64])
@@ -448,7 +421,7 @@ def test_moe_layer_stages_vs_oracle():
     assert_combine_close(out, oracle.moe_combine(yb, i_ref, p["tw"]), yb, i_ref, p["tw"])
 
 
-@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
+@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA])
 @pytest.mark.parametrize("dtype", [INT8, FP8])
 def test_grouped_gemm_tcgen05_vs_oracle(path, dtype):
     p = moe_problem(T=300, H=384, I=256, E=8, dtype=dtype, seed=33)
@@ -545,7 +518,7 @@ def test_fused_w13_silu_requant_rows_past_offsets_and_paths():
                                    dev_u8(p2["q13"]), dev_f32(p2["s13"]), INT8)
     assert ei.value.status == bq.ERR_UNSUPPORTED
     # only the tensor-core path has the fused epilogue
-    for path in (bq.PATH_SIMT, bq.PATH_TCGEN05_2CTA):
+    for path in (bq.PATH_SIMT,):
         bq.set_path(path)
         with pytest.raises(bq.BqError) as ei:
             bq.grouped_gemm_silu_quant(qa, sa, dev_i32(off), dev_u8(p["q13"]),
@@ -554,7 +527,7 @@ def test_fused_w13_silu_requant_rows_past_offsets_and_paths():
     bq.set_path(bq.PATH_AUTO)
 
 
-@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_2CTA])
+@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05_1CTA])
 def test_grouped_gemm_leaves_rows_past_offsets_untouched(path):
     p = moe_problem(T=50, H=128, I=128, E=4)
     bq.set_path(path)
@@ -771,3 +744,73 @@ def test_mx_gemm_narrow_n_and_strided_operands():
     torch.cuda.synchronize()
     bq.check_device_status()
     assert_gemm_close(out, oracle.mx_gemm(qa, sa, qw, sw), "MXFP8 strided operands")
+
+
+# --------------------------------------------------------------------------
+# K-sharded (row-parallel) linear: fp32 partials, one rounding at the end
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", [bq.PATH_AUTO, bq.PATH_SIMT])
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+@pytest.mark.parametrize("M,N,K,shards", [(1, 4096, 4096, 2),    # cluster decode kernel
+                                          (37, 1000, 1536, 3),   # decode, ragged N
+                                          (300, 640, 1024, 2),   # tcgen05 kernel
+                                          (200, 256, 896, 7)])
+def test_gemm_partial_shards_sum_then_round_once(path, dtype, M, N, K, shards):
+    _, qa, sa, qw, sw, bb = make_problem(M, N, K, 128, 128, dtype, 800 + M, bias=True)
+    bq.set_path(path)
+    kb = K // 128 // shards
+    edges = [128 * kb * i for i in range(shards)] + [K]
+    total = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    for a, b in zip(edges[:-1], edges[1:]):
+        part = bq.gemm_partial(dev_u8(np.ascontiguousarray(qa[:, a:b])),
+                               dev_f32(np.ascontiguousarray(sa[:, a // 128:b // 128].T)),
+                               dev_u8(np.ascontiguousarray(qw[:, a:b])),
+                               dev_f32(np.ascontiguousarray(sw[:, a // 128:b // 128])),
+                               128, 128, dtype)
+        total += part                                  # the all-reduce, on one GPU
+    out = bq.finish_bf16(total, dev_bf16(bb))
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    ref = oracle.gemm(qa, sa, qw, sw, 128, 128, dtype, bias_bf16=bb)
+    assert_gemm_close(out, ref, f"sharded x{shards} {M}x{N}x{K} dtype={dtype}")
+
+
+def test_finish_bf16_rounds_the_fp32_sum_once():
+    rng = np.random.default_rng(5)
+    for M, N in ((3, 7), (64, 4096), (5, 1001)):
+        part = torch.from_numpy(rng.normal(0, 3, (M, N)).astype(np.float32))
+        bias = torch.from_numpy(rng.normal(0, 1, N).astype(np.float32)).to(torch.bfloat16)
+        out = bq.finish_bf16(part.cuda(), bias.cuda())
+        torch.cuda.synchronize()
+        # the fp32 add, then torch's round-to-nearest-even conversion
+        ref = (part + bias.float()[None, :]).to(torch.bfloat16)
+        assert torch.equal(out.cpu().view(torch.int16), ref.view(torch.int16))
+        out = bq.finish_bf16(part.cuda())
+        assert torch.equal(out.cpu().view(torch.int16), part.to(torch.bfloat16).view(torch.int16))
+
+
+def test_tensor_parallel_layers_on_one_rank_use_the_cuda_kernels():
+    """tp.py on a one-rank group (no collective runs): the CUDA backend's
+    column- and row-parallel layers equal the unsharded layer."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from block_scaled_w8a8_b200 import tp
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        xb, qa, sa, qw, sw, bb = make_problem(24, 512, 768, 128, 128, INT8, 61, bias=True)
+        x, qwd, swd, bias = dev_bf16(xb), dev_u8(qw), dev_f32(sw), dev_bf16(bb)
+        ycol = tp.column_parallel_linear(x, qwd, swd, bias)
+        yrow = tp.row_parallel_linear(x, qwd, swd, bias)
+        torch.cuda.synchronize()
+        bq.check_device_status()
+        ref = oracle.gemm(qa, sa, qw, sw, 128, 128, INT8, bias_bf16=bb)
+        assert_gemm_close(ycol, ref, "column parallel, one rank")
+        assert_gemm_close(yrow, ref, "row parallel, one rank")
+    finally:
+        dist.destroy_process_group()

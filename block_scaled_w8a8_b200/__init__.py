@@ -57,6 +57,7 @@ DECLS = {
     "bq_linear_workspace_size": (_INT, [_I64, _I64, _I64, _I64, _I64, _INT, _SZP]),
     "bq_linear": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I64, _I64, _INT, _P, _P,
                          _I64, _P, _SZ, _P]),
+    "bq_moe_route": (_INT, [_P, _I64, _I64, _I64, _I64, _P, _P, _P]),
     "bq_moe_permute_workspace_size": (_INT, [_I64, _I64, _I64, _SZP]),
     "bq_moe_permute": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "bq_moe_quant_gather": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _I64, _INT, _P, _I64, _P,
@@ -302,6 +303,21 @@ def linear(x, qw, sw, block_n=128, block_k=128, dtype=INT8, bias=None, out=None,
                            _cuda(out, "out"), _ld(out), _opt(ws, "ws"),
                            0 if ws is None else ws.numel(), _P(_stream(x.device))))
     return out
+
+
+def moe_route(logits: torch.Tensor, topk: int, ids=None, weights=None):
+    """Top-k experts of fp32 router logits [T, E] and their renormalised
+    softmax weights -> (ids int32 [T, topk], weights float32 [T, topk])."""
+    assert logits.dtype == torch.float32
+    T, E = logits.shape
+    if ids is None:
+        ids = torch.empty(T, topk, dtype=torch.int32, device=logits.device)
+    if weights is None:
+        weights = torch.empty(T, topk, dtype=torch.float32, device=logits.device)
+    _check(lib().bq_moe_route(_cuda(logits, "logits"), _ld(logits), T, E, topk,
+                              _cuda(ids, "ids"), _cuda(weights, "weights"),
+                              _P(_stream(logits.device))))
+    return ids, weights
 
 
 def moe_permute(topk_ids: torch.Tensor, E: int):

@@ -408,6 +408,21 @@ bq_status bq_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void
                    base, g, stream, true);
 }
 
+bq_status bq_moe_route(const float* logits, int64_t ld, int64_t T, int64_t E, int64_t topk,
+                       int32_t* topk_ids, float* topk_weights, void* stream) {
+  BQ_CHECK_ARG(T >= 0 && E >= 1 && topk >= 1, "need T >= 0, E >= 1, topk >= 1");
+  BQ_CHECK_ARG(topk <= E, "topk (%lld) exceeds E (%lld)", (long long)topk, (long long)E);
+  BQ_CHECK_ARG(ld >= E, "ld must be >= E");
+  if (E > 256 || topk > 8)
+    return fail(BQ_ERR_UNSUPPORTED, "routing supports E <= 256 and topk <= 8");
+  if (T == 0) return ok();
+  BQ_CHECK_ARG(logits && topk_ids && topk_weights, "logits, ids and weights must not be NULL");
+  BQ_CHECK_CUDA(bq::launch_moe_route(logits, ld, T, E, topk, topk_ids, topk_weights,
+                                     as_stream(stream)),
+                "moe_route launch");
+  return ok();
+}
+
 bq_status bq_moe_permute_workspace_size(int64_t T, int64_t topk, int64_t E, size_t* bytes) {
   BQ_CHECK_ARG(T >= 0 && topk >= 1 && E >= 1, "need T >= 0, topk >= 1, E >= 1");
   BQ_CHECK_ARG(bytes, "bytes must not be NULL");

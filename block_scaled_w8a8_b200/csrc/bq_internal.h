@@ -63,6 +63,10 @@ cudaError_t launch_moe_combine(const void* y, int64_t ldy, const int32_t* inv_pe
 cudaError_t launch_finish_bf16(const float* part, int64_t ldp, int64_t M, int64_t N,
                                const void* bias, void* out, int64_t ldo, cudaStream_t st);
 
+// Top-k routing from fp32 router logits [T, E] (row stride ld).
+cudaError_t launch_moe_route(const float* logits, int64_t ld, int64_t T, int64_t E,
+                             int64_t topk, int32_t* ids, float* w, cudaStream_t st);
+
 // Bounded-wait self-test.
 cudaError_t launch_selftest_wait(int64_t spin_limit, unsigned* status, cudaStream_t st);
 

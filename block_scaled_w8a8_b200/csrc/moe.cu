@@ -11,6 +11,14 @@
 //
 // Combine: out[t, n] = bf16( sum_j w[t, j] * y[inv_perm[t*topk+j], n] ),
 // fp32 accumulation, one rounding; 8 bf16 per thread with 16-byte vectors.
+//
+// Routing (the topk_ids / topk_weights the MoE runner of sections 5-6
+// receives): one warp per token picks its top-k experts from the fp32 router
+// logits -- the softmax is monotonic, so the k largest logits are the k
+// largest probabilities, ties to the lower expert index -- and weights them
+// exp(l_j - l_max) / sum over the k of exp(l_i - l_max): the softmax
+// probabilities renormalised over the chosen k (the full softmax denominator
+// cancels).
 #include <algorithm>
 
 #include "bq_common.cuh"
@@ -130,6 +138,64 @@ moe_combine_kernel(const uint16_t* __restrict__ y, int64_t ldy,
 
 // Waits for a flag that nothing sets, at most spin_limit polls, then records
 // a timeout in the status word and returns.
+constexpr int kRouteMaxE = 256, kRouteMaxK = 8;
+
+__global__ void __launch_bounds__(256)
+moe_route_kernel(const float* __restrict__ logits, int64_t ld, int64_t T, int E, int topk,
+                 int32_t* __restrict__ ids, float* __restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kRouteMaxE / 32;
+  const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + t * ld;
+  // lane holds experts lane, lane + 32, ...
+  float v[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? row[e] : -INFINITY;
+  }
+  unsigned taken = 0;                           // bit i: expert lane + 32 i chosen
+  int sel[kRouteMaxK];
+  float lsel[kRouteMaxK];
+  for (int j = 0; j < topk; ++j) {
+    // this lane's best unchosen (largest logit, then lowest expert index)
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !(taken & (1u << i)) && (v[i] > bv || (v[i] == bv && e < be))) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    sel[j] = be;
+    lsel[j] = bv;
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+  }
+  if (lane == 0) {
+    float ex[kRouteMaxK], sum = 0.0f;
+    for (int j = 0; j < topk; ++j) {
+      ex[j] = expf(lsel[j] - lsel[0]);
+      sum += ex[j];
+    }
+    for (int j = 0; j < topk; ++j) {
+      ids[t * topk + j] = sel[j];
+      w[t * topk + j] = ex[j] / sum;
+    }
+  }
+}
+
 __global__ void selftest_wait_kernel(int64_t spin_limit, unsigned* status) {
   __shared__ volatile int flag;
   if (threadIdx.x == 0) flag = 0;
@@ -168,6 +234,17 @@ cudaError_t launch_moe_combine(const void* y, int64_t ldy, const int32_t* inv_pe
   moe_combine_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(y), ldy, inv_perm, w, T,
                                            (int)topk, H, static_cast<uint16_t*>(out), ldo,
                                            vec);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_moe_route(const float* logits, int64_t ld, int64_t T, int64_t E,
+                             int64_t topk, int32_t* ids, float* w, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (E < 1 || E > kRouteMaxE || topk < 1 || topk > kRouteMaxK || topk > E)
+    return cudaErrorInvalidValue;
+  const int64_t blocks = (T + 7) / 8;
+  if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+  moe_route_kernel<<<(unsigned)blocks, 256, 0, st>>>(logits, ld, T, (int)E, (int)topk, ids, w);
   return cudaGetLastError();
 }
 

@@ -124,14 +124,19 @@ def linear_inputs(cfg: Linear, device="cpu"):
     return a, w
 
 
+def router_logits(T: int, E: int, seed: int) -> torch.Tensor:
+    """The router logits of the MoE workload: fp32 [T, E] ~ N(0, 1) (CPU)."""
+    g = _gen(seed + 7919, "cpu")
+    return torch.randn(T, E, generator=g, dtype=torch.float32)
+
+
 def routing(T: int, E: int, topk: int, seed: int):
     """Top-k routing from softmax of N(0,1) logits (harness choice).
 
     Softmax in fp64; experts ranked by probability, ties to the lower index;
     the top-k probabilities are renormalised to sum to one.  Returns
     (ids int32 [T, topk], weights float32 [T, topk]) as numpy arrays."""
-    g = _gen(seed + 7919, "cpu")
-    logits = torch.randn(T, E, generator=g, dtype=torch.float32).double().numpy()
+    logits = router_logits(T, E, seed).double().numpy()
     z = logits - logits.max(axis=1, keepdims=True)
     p = np.exp(z)
     p /= p.sum(axis=1, keepdims=True)

@@ -282,6 +282,19 @@ bq_status bq_linear(const void* x, int64_t ldx, int64_t M, int64_t K, const void
 
 /* ---- MoE (block-wise INT8 page, sections 5 and 6) ---------------- */
 
+/* Top-k routing of T tokens over E experts from fp32 router logits [T, E]
+ * (row stride ld >= E): topk_ids int32 [T, topk] are the experts of the topk
+ * largest logits of each row, in descending order, ties to the lower expert
+ * index (the softmax is monotonic, so these are the topk most probable
+ * experts); topk_weights fp32 [T, topk] are their softmax probabilities
+ * renormalised over the chosen topk, computed as exp(l_j - l_max) divided by
+ * the sum over the topk (fp32 expf: within a few ulp of the exact values).
+ * These are the topk_ids / topk_weights the MoE runner of the block-wise INT8
+ * page (sections 5-6) receives; the pages leave the tie order and the
+ * renormalisation open, and this is the reading taken.  E <= 256, topk <= 8. */
+bq_status bq_moe_route(const float* logits, int64_t ld, int64_t T, int64_t E, int64_t topk,
+                       int32_t* topk_ids, float* topk_weights, void* stream);
+
 /* Bytes of workspace bq_moe_permute needs. */
 bq_status bq_moe_permute_workspace_size(int64_t T, int64_t topk, int64_t E, size_t* bytes);
 

@@ -107,6 +107,8 @@ def configure(lib):
     lib.bq_ref_mx_quant.restype = None
     lib.bq_ref_mx_gemm.argtypes = [P, L, P, P, L, P, L, L, L, P, P]
     lib.bq_ref_mx_gemm.restype = None
+    lib.bq_ref_moe_route.argtypes = [P, L, L, L, L, P, P]
+    lib.bq_ref_moe_route.restype = None
     lib.bq_ref_threads.argtypes = [I]
     lib.bq_ref_threads.restype = I
     return lib
@@ -278,6 +280,20 @@ def dequant_dot(qa, sa, qw, sw, bn: int, bk: int, dtype: int, m: int, n: int,
 # --------------------------------------------------------------------------
 # MoE
 # --------------------------------------------------------------------------
+
+def moe_route(logits: np.ndarray, topk: int):
+    """Top-k routing of each row of fp32 logits [T, E]: softmax in fp64,
+    experts by descending probability (ties to the lower index), the top-k
+    probabilities renormalised to sum to one.  Returns (ids int32 [T, topk],
+    weights float32 [T, topk])."""
+    lib = _load()
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    ids = np.empty((T, topk), dtype=np.int32)
+    w = np.empty((T, topk), dtype=np.float32)
+    lib.bq_ref_moe_route(_ptr(lg), E, T, E, topk, _ptr(ids), _ptr(w))
+    return ids, w
+
 
 def moe_permute(ids: np.ndarray, E: int):
     """Stable expert-major order of the (token, slot) pairs.

@@ -303,6 +303,50 @@ double bq_ref_dequant_dot(const uint8_t* qa, long lda, const float* sa, const ui
 }
 
 /* ------------------------------------------------------------------------ */
+/* MoE routing: topk_ids and topk_weights, the inputs the block-wise INT8  */
+/* page's MoE runner (§5-§6) receives; the workload routes each token to   */
+/* its top-2 experts by the softmax of its router logits.  The pages do    */
+/* not fix the tie order or whether the top-k weights are renormalised;    */
+/* the reading: softmax in fp64, experts by descending probability, ties   */
+/* to the lower expert index, the k probabilities divided by their sum.    */
+/* ------------------------------------------------------------------------ */
+
+/* logits: fp32 [T, E] (row stride ld); ids: int32 [T, topk]; w: fp32 [T, topk]. */
+void bq_ref_moe_route(const float* logits, long ld, long T, long E, long topk, int32_t* ids,
+                      float* w) {
+    double* p = (double*)malloc(sizeof(double) * (size_t)(E > 0 ? E : 1));
+    unsigned char* taken = (unsigned char*)malloc((size_t)(E > 0 ? E : 1));
+    for (long t = 0; t < T; t++) {
+        const float* l = logits + t * ld;
+        double mx = (double)l[0];
+        for (long e = 1; e < E; e++)
+            if ((double)l[e] > mx) mx = (double)l[e];
+        double sum = 0.0;
+        for (long e = 0; e < E; e++) {
+            p[e] = exp((double)l[e] - mx);
+            sum += p[e];
+        }
+        for (long e = 0; e < E; e++) {
+            p[e] /= sum;
+            taken[e] = 0;
+        }
+        double topsum = 0.0;
+        for (long j = 0; j < topk; j++) {
+            long best = -1;
+            for (long e = 0; e < E; e++)
+                if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+            taken[best] = 1;
+            ids[t * topk + j] = (int32_t)best;
+            topsum += p[best];
+        }
+        for (long j = 0; j < topk; j++)
+            w[t * topk + j] = (float)(p[ids[t * topk + j]] / topsum);
+    }
+    free(p);
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------ */
 /* MoE token permutation ([BWI8] §5-§6: per-expert weights, routed      */
 /* tokens).  Stable order: by expert, then by flat slot index t*topk + j.   */
 /* ------------------------------------------------------------------------ */

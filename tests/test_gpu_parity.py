@@ -814,3 +814,31 @@ def test_tensor_parallel_layers_on_one_rank_use_the_cuda_kernels():
         assert_gemm_close(yrow, ref, "row parallel, one rank")
     finally:
         dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# device-side routing
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,topk", [(4096, 8, 2), (37, 8, 1), (300, 64, 6), (5, 256, 8),
+                                      (100, 3, 3), (33, 40, 2)])
+def test_moe_route_vs_oracle(T, E, topk):
+    lg = bq_synth.router_logits(T, E, 100 + E).numpy()
+    lg[: T // 3, E // 2] = lg[: T // 3, 0]            # exact ties: the lower index wins
+    ids, w = bq.moe_route(torch.from_numpy(lg).cuda(), topk)
+    torch.cuda.synchronize()
+    ids_ref, w_ref = oracle.moe_route(lg, topk)
+    # the experts come from comparing the same fp32 logits: bit-exact
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    # fp32 expf, sum and division against the fp64 softmax: a few fp32 ulp
+    np.testing.assert_allclose(w.cpu().numpy(), w_ref, rtol=2e-6, atol=1e-7)
+
+
+def test_moe_route_rejects_out_of_range_shapes():
+    lg = torch.zeros(4, 300, device="cuda")
+    with pytest.raises(bq.BqError) as ei:
+        bq.moe_route(lg, 2)
+    assert ei.value.status == bq.ERR_UNSUPPORTED
+    with pytest.raises(bq.BqError) as ei:
+        bq.moe_route(torch.zeros(4, 4, device="cuda"), 5)
+    assert ei.value.status == bq.ERR_INVALID_ARG

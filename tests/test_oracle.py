@@ -567,30 +567,36 @@ def test_mx_quant_invariants_over_a_wide_range():
     assert np.all(np.abs(deq[sat]) == 448 * scale[sat])
 
 
-def test_threaded_build_computes_the_same_results():
-    # the OpenMP build only splits rows over threads (used to time the CPU
-    # baseline on all host cores): every output is bit-identical to the
-    # single-threaded build's
-    rng = np.random.default_rng(31)
-    M, N, K = 37, 300, 520
-    xb = oracle.bf16_from_f64(rng.normal(0, 1, (M, K)))
-    w = rng.normal(0, 0.02, (N, K))
-    y = oracle.bf16_from_f64(rng.normal(0, 1, (24, 2 * 96)))
-    inv = rng.permutation(24).astype(np.int32)
-    tw = rng.random(24).astype(np.float32)
-    results = []
-    for threads in (1, 4):
-        oracle.use_threads(threads)
-        try:
-            qa, sa = oracle.quant_act(xb, 128, oracle.INT8)
-            qw, sw = oracle.quant_weight(w, 128, 128, oracle.INT8)
-            o64 = oracle.gemm(qa, sa, qw, sw, 128, 128, oracle.INT8)
-            h = oracle.silu_mul(y, 96)
-            c = oracle.moe_combine(y, inv, tw.reshape(12, 2))
-            mq, ms = oracle.mx_quant(w[:5, :512])
-            mo = oracle.mx_gemm(mq, ms, mq, ms)
-            results.append((qa, sa, qw, sw, o64, h, c, mo))
-        finally:
-            oracle.use_threads(1)
-    for a, b in zip(*results):
-        assert np.array_equal(a, b)
+
+# --------------------------------------------------------------------------
+# MoE routing (top-k of the softmax of router logits)
+# --------------------------------------------------------------------------
+
+def test_route_hand_worked():
+    # logits 0 and ln 3: probabilities 1/4 and 3/4
+    lg = np.array([[0.0, np.log(3.0)]], np.float32)
+    ids, w = oracle.moe_route(lg, 2)
+    assert ids.tolist() == [[1, 0]]
+    np.testing.assert_allclose(w, [[0.75, 0.25]], rtol=1e-6)
+    ids, w = oracle.moe_route(lg, 1)
+    assert ids.tolist() == [[1]] and w.tolist() == [[1.0]]
+    # equal logits: the lower expert index first
+    ids, _ = oracle.moe_route(np.array([[2.0, 5.0, 5.0, 5.0, -1.0]], np.float32), 3)
+    assert ids.tolist() == [[1, 2, 3]]
+
+
+def test_route_matches_a_stable_argsort_of_the_fp64_softmax():
+    rng = np.random.default_rng(17)
+    lg = rng.normal(0, 1, (300, 8)).astype(np.float32)
+    lg[:20, 3] = lg[:20, 5]                          # exact ties
+    for topk in (1, 2, 3, 8):
+        ids, w = oracle.moe_route(lg, topk)
+        z = lg.astype(np.float64)
+        p = np.exp(z - z.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        order = np.argsort(-p, axis=1, kind="stable")[:, :topk]
+        assert np.array_equal(ids, order)
+        top = np.take_along_axis(p, order, axis=1)
+        np.testing.assert_allclose(w, top / top.sum(axis=1, keepdims=True), rtol=1e-6)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-6)
+        assert np.all(np.diff(w, axis=1) <= 0)       # descending weights

@@ -46,6 +46,10 @@ MUTANTS = {
     "mx_bias_dropped": ("if (bias != NULL) acc += bq_ref_bf16_to_double(bias[n]);", ""),
     "mx_act_scale_first_group_only": ("ldexp(1.0, (int)sa[m * G + g] - 127)",
                                       "ldexp(1.0, (int)sa[m * G] - 127)"),
+    "route_ties_to_higher_index": ("if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;",
+                                   "if (!taken[e] && (best < 0 || p[e] >= p[best])) best = e;"),
+    "route_not_renormalised": ("w[t * topk + j] = (float)(p[ids[t * topk + j]] / topsum);",
+                               "w[t * topk + j] = (float)(p[ids[t * topk + j]]);"),
     "bf16_ties_up": ("else r = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;\n    double res",
                      "else r = f + 1.0;\n    double res"),
 }

@@ -449,23 +449,26 @@ def bench_tiny(args, dist, bq, stream):
 
 class MoeLayer:
     """The MoE layer of the block-int8 MoE workload (T tokens, E experts, top-k),
-    device-resident: routing, block-quantised w13 / w2, every intermediate,
-    and run(parts) that enqueues the layer's library calls in order.  The
-    full-size parity test drives the same object.  The layer as timed fuses
-    the w13 GEMM with silu * up and its requantisation ("w13silu"); the
-    unfused parts ("w13", "silu") store and re-read the bf16 w13 output."""
+    device-resident: router logits, block-quantised w13 / w2, every
+    intermediate, and run(parts) that enqueues the layer's library calls in
+    order.  The full-size parity test drives the same object.  The layer as
+    timed routes on the device ("route": softmax top-k of the logits), fuses
+    the w13 GEMM with silu * up and its requantisation ("w13silu"), and the
+    w2 GEMM with the weighted top-k combine ("w2comb": fp32 atomic sums into
+    token rows, then "fin" rounds them once to bf16).  The unfused parts
+    ("w13", "silu", "w2", "comb") store and re-read the bf16 intermediates."""
 
-    PARTS = ("perm", "gather", "w13silu", "w2", "comb")
-    UNFUSED = ("perm", "gather", "w13", "silu", "w2", "comb")
+    PARTS = ("route", "perm", "gather", "w13silu", "w2comb", "fin")
+    UNFUSED = ("route", "perm", "gather", "w13", "silu", "w2", "comb")
 
     def __init__(self, bq, dev, cfg=None):
         cfg = cfg or bq_synth.MOE
         self.bq, self.cfg = bq, cfg
         T, H, I, E, topk = cfg.T, cfg.H, cfg.I, cfg.E, cfg.topk
         self.x = bq_synth.activations(T, H, cfg.seed, device=dev)
-        self.ids, self.tw = bq_synth.routing(T, E, topk, cfg.seed)
-        self.ids_d = torch.from_numpy(self.ids).to(dev)
-        self.tw_d = torch.from_numpy(self.tw).to(dev)
+        self.logits = bq_synth.router_logits(T, E, cfg.seed).to(dev)
+        self.ids_d = torch.empty(T, topk, dtype=torch.int32, device=dev)
+        self.tw_d = torch.empty(T, topk, dtype=torch.float32, device=dev)
         self.q13 = torch.empty(E, 2 * I, H, dtype=torch.uint8, device=dev)
         self.s13 = torch.empty(E, 2 * cdiv(I, 128), cdiv(H, 128), dtype=torch.float32,
                                device=dev)
@@ -491,6 +494,7 @@ class MoeLayer:
         self.qh = torch.empty(R, I, dtype=torch.uint8, device=dev)
         self.sh = torch.empty(cdiv(I, 128), R, dtype=torch.float32, device=dev)
         self.y2 = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+        self.acc = torch.zeros(T, H, dtype=torch.float32, device=dev)   # "fin" re-zeroes it
         self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.ws = bq.workspace(bq.grouped_gemm_workspace_size(R, 2 * I, H, E), dev)
         torch.cuda.synchronize()
@@ -507,6 +511,8 @@ class MoeLayer:
         bq, c = self.bq, self.cfg
         L = bq.lib()
         st = torch.cuda.current_stream().cuda_stream
+        if "route" in parts:
+            bq.moe_route(self.logits, c.topk, ids=self.ids_d, weights=self.tw_d)
         if "perm" in parts:
             bq._check(L.bq_moe_permute(self.ids_d.data_ptr(), c.T, c.topk, c.E,
                                        self.off.data_ptr(), self.perm.data_ptr(),
@@ -524,6 +530,11 @@ class MoeLayer:
         if "w2" in parts:
             bq.grouped_gemm(self.qh, self.sh, self.off, self.q2, self.s2, 128, 128, 0, c.dtype,
                             out=self.y2, ws=self.ws)
+        if "w2comb" in parts:
+            bq.grouped_gemm_combine(self.qh, self.sh, self.off, self.q2, self.s2, self.perm,
+                                    self.tw_d, self.acc, c.dtype)
+        if "fin" in parts:
+            bq.moe_combine_finish(self.acc, out=self.out)
         if "comb" in parts:
             bq.moe_combine(self.y2, self.inv, self.tw_d, out=self.out)
 
@@ -539,24 +550,28 @@ def bench_moe(args, dist, bq, peaks, stream):
         return lambda: moe.run(parts)
 
     g = [capture(layer(), stream)]
-    gg = [capture(layer(("w13silu", "w2")), stream)]
+    gg = [capture(layer(("w13silu", "w2comb")), stream)]
+    gu = [capture(layer(MoeLayer.UNFUSED), stream)]
     steps = max(3, args.steps // 4)
     with Clocks(torch.cuda.current_device()) as clk:
         t = timed_graph_steps(g, steps, args.warmup, stream, dist)
         t_g = timed_graph_steps(gg, steps, args.warmup, stream, dist)
+        t_u = timed_graph_steps(gu, steps, args.warmup, stream, dist)
     ops = 2.0 * R * (2 * I) * H + 2.0 * R * H * I
     peak = 2.0 * peaks["bf16_tflops"]
     ach = ops / (t_g / steps) / 1e12
-    del g, gg
+    del g, gg, gu
     return {"value": whole_job_rate(dist.world, steps, ops, t) / 1e12, "unit": "TOPS",
             "ms_per_step": 1e3 * t / steps, "steps": steps,
+            "unfused_ms_per_step": 1e3 * t_u / steps,
             "roofline": {"bound": "tensor",
-                         "kernel": "tcgen05 grouped GEMM (w13 fused with silu*up requant, + w2)",
+                         "kernel": "tcgen05 grouped GEMMs (w13 fused with silu*up requant, "
+                                   "w2 fused with the weighted combine)",
                          "achieved": ach, "peak": peak, "unit": "TOPS", "frac": ach / peak,
                          "traffic": None, "avg_pair_us": 1e6 * t_g / steps},
             "clocks": clk.summary(),
             "config": {"workload": cfg.name, "T": T, "H": H, "I": I, "E": E, "topk": topk,
-                       "block": [128, 128], "routing": "softmax(N(0,1) logits) top-2"},
+                       "block": [128, 128], "routing": "device softmax top-2 of N(0,1) logits"},
             "dtype": "int8"}
 
 
@@ -690,7 +705,10 @@ def cpu_baseline_moe(seconds_target=4.0):
     threads = oracle.use_threads(hi["nproc"])
     try:
         T, H, I, E, topk = cfg.T, cfg.H, cfg.I, cfg.E, cfg.topk
-        ids, tw = bq_synth.routing(T, E, topk, cfg.seed)
+        logits = bq_synth.router_logits(T, E, cfg.seed).numpy()
+        t0 = time.perf_counter()
+        ids, tw = oracle.moe_route(logits, topk)
+        t_route = time.perf_counter() - t0
         rows = max(2 * threads, 8)
         # a sample of the expert's intermediate width: I2 gate rows, the
         # matching up rows, and the w2 columns they feed
@@ -711,6 +729,7 @@ def cpu_baseline_moe(seconds_target=4.0):
             out = fn()
             return out, time.perf_counter() - t0
 
+        stages["route"] = {"value": T / t_route / 1e6, "unit": "M tokens/s"}
         (_, _, _), t_perm = timed(lambda: oracle.moe_permute(ids, E))
         stages["permute"] = {"value": T * topk / t_perm / 1e6, "unit": "M pairs/s"}
         tot_gemm, tot_t = 0.0, 0.0
@@ -735,7 +754,7 @@ def cpu_baseline_moe(seconds_target=4.0):
         oracle.use_threads(1)
     return {"value": tot_gemm / tot_t / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
             "stages": stages,
-            "sample": f"permute of all {T * topk} pairs; expert 0 with {rows} token rows and "
+            "sample": f"routing of all {T} tokens; permute of all {T * topk} pairs; expert 0 with {rows} token rows and "
                       f"{I} of its {cfg.I} intermediate columns through quant, w13, silu*up + "
                       f"requant, w2 and combine; C oracle on {threads} threads; {tot_t:.1f} s"}
 

@@ -67,6 +67,9 @@ DECLS = {
                                _I64, _INT, _P, _I64, _P, _SZ, _P]),
     "bq_grouped_gemm_silu_quant": (_INT, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64,
                                           _I64, _I64, _INT, _P, _I64, _P, _P]),
+    "bq_grouped_gemm_combine": (_INT, [_P, _I64, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _I64,
+                                       _I64, _INT, _P, _P, _I64, _P, _I64, _P]),
+    "bq_moe_combine_finish": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P]),
     "bq_moe_silu_mul_quant": (_INT, [_P, _I64, _I64, _I64, _I64, _INT, _P, _I64, _P, _P, _P]),
     "bq_mx_scale_bytes": (_INT, [_I64, _I64, _SZP]),
     "bq_mx_quant_act": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _P]),
@@ -393,6 +396,34 @@ def grouped_gemm_silu_quant(qa, sa, offsets, qw13, sw13, dtype=INT8, q=None, s=N
                                             _cuda(q, "q"), _ld(q), _cuda(s, "s"),
                                             _P(_stream(qa.device))))
     return q, s
+
+
+def grouped_gemm_combine(qh, sh, offsets, qw2, sw2, perm, topk_w, acc, dtype=INT8):
+    """w2 grouped GEMM fused with the weighted top-k combine: adds
+    topk_w[perm[r]] * bf16(row r of the GEMM) into fp32 acc [T, N] row
+    perm[r] // topk.  acc must hold zeros on entry; moe_combine_finish rounds
+    it to bf16 and zeroes it."""
+    R, K = qh.shape
+    E, N, _ = qw2.shape
+    T, topk = topk_w.shape
+    assert acc.dtype == torch.float32 and acc.shape[0] == T and acc.shape[1] >= N
+    assert qw2.is_contiguous() and sw2.is_contiguous() and topk_w.is_contiguous()
+    _check(lib().bq_grouped_gemm_combine(_cuda(qh, "qh"), _ld(qh), _cuda(sh, "sh"), R,
+                                         _cuda(offsets, "offsets"), E, _cuda(qw2, "qw2"),
+                                         _cuda(sw2, "sw2"), N, K, 128, 128, dtype,
+                                         _cuda(perm, "perm"), _cuda(topk_w, "topk_w"), topk,
+                                         _cuda(acc, "acc"), _ld(acc), _P(_stream(qh.device))))
+    return acc
+
+
+def moe_combine_finish(acc, out=None):
+    """bf16(acc) into out [T, N]; acc is zeroed."""
+    T, N = acc.shape
+    if out is None:
+        out = torch.empty(T, N, dtype=torch.bfloat16, device=acc.device)
+    _check(lib().bq_moe_combine_finish(_cuda(acc, "acc"), T, N, _ld(acc), _cuda(out, "out"),
+                                       _ld(out), _P(_stream(acc.device))))
+    return out
 
 
 def mx_scale_bytes(R, K):

@@ -550,6 +550,55 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
   return ok();
 }
 
+bq_status bq_grouped_gemm_combine(const void* qa, int64_t lda, const float* sa, int64_t R,
+                                  const int32_t* expert_offsets, int64_t E, const void* qw,
+                                  const float* sw, int64_t N, int64_t K, int64_t block_n,
+                                  int64_t block_k, int dtype, const int32_t* perm,
+                                  const float* topk_w, int64_t topk, float* acc, int64_t ld_acc,
+                                  void* stream) {
+  bq_status st = check_gemm_shape(R, N, K, block_n, block_k, dtype);
+  if (st != BQ_OK) return st;
+  BQ_CHECK_ARG(E >= 1 && E <= 65535, "E must be in [1, 65535]");
+  BQ_CHECK_ARG(topk >= 1 && topk <= 65535, "topk must be in [1, 65535]");
+  BQ_CHECK_ARG(R % topk == 0, "R must be T * topk");
+  BQ_CHECK_ARG(lda >= K && ld_acc >= N, "leading dimensions too small");
+  if (R == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(acc && perm && topk_w && expert_offsets,
+               "acc, perm, topk_w and expert_offsets must not be NULL");
+  BQ_CHECK_ARG(K == 0 || (qa && sa && qw && sw), "qa, sa, qw and sw must not be NULL");
+  if (!(g_path == BQ_PATH_AUTO || g_path == BQ_PATH_TCGEN05 || g_path == BQ_PATH_TCGEN05_1CTA))
+    return fail(BQ_ERR_UNSUPPORTED, "the combining GEMM runs on the tensor-core path only");
+  const int64_t Kb = cdiv(K, block_k);
+  bq::GemmArgs a{};
+  a.qa = qa; a.lda = lda; a.sa = sa; a.sa_rows = R;
+  a.qw = qw; a.ldw = K; a.sw = sw;
+  a.M = R; a.N = N; a.K = K; a.bn = block_n; a.bk = block_k; a.seam = 0;
+  a.Nbs = cdiv(N, block_n);
+  a.dtype = dtype; a.bias = nullptr; a.out = nullptr; a.ldo = ld_acc;
+  a.offsets = expert_offsets; a.E = E;
+  a.w_expert_stride = N * K; a.sw_expert_stride = a.Nbs * Kb;
+  a.comb_acc = acc; a.comb_perm = perm; a.comb_w = topk_w; a.topk = topk;
+  char why[256] = "";
+  if (!bq::tc_supported(a, why, sizeof(why))) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
+  unsigned* w = nullptr;
+  st = status_word(&w);
+  if (st != BQ_OK) return st;
+  a.status = w;
+  BQ_CHECK_CUDA(bq::launch_gemm_tc(a, as_stream(stream)), "combining grouped GEMM launch");
+  return ok();
+}
+
+bq_status bq_moe_combine_finish(float* acc, int64_t T, int64_t N, int64_t ld_acc, void* out,
+                                int64_t ldo, void* stream) {
+  BQ_CHECK_ARG(T >= 0 && N >= 0, "need T >= 0 and N >= 0");
+  BQ_CHECK_ARG(ld_acc >= N && ldo >= N, "leading dimensions must be >= N");
+  if (T == 0 || N == 0) return ok();
+  BQ_CHECK_ARG(acc && out, "acc and out must not be NULL");
+  BQ_CHECK_CUDA(bq::launch_moe_combine_finish(acc, T, N, ld_acc, out, ldo, as_stream(stream)),
+                "moe_combine_finish launch");
+  return ok();
+}
+
 // ---------------- MXFP8 ----------------
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }

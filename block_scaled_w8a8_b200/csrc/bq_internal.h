@@ -47,6 +47,10 @@ struct GemmArgs {
   // fp32 partial output (bq_gemm_partial): when set, out and bias are unused
   // and the kernel stores sum_kb P_kb * sa * sw unrounded to out_f32 [M, ldo]
   float* out_f32;
+  // weighted top-k combine (tcgen05 path only): when comb_acc is set, out
+  // and bias are unused and row m adds comb_w[comb_perm[m]] * bf16(row m) to
+  // fp32 row comb_perm[m] / topk of comb_acc (row stride ldo) atomically
+  float* comb_acc; const int32_t* comb_perm; const float* comb_w; int64_t topk;
 };
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
@@ -55,6 +59,9 @@ cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);
 cudaError_t launch_moe_permute(const int32_t* ids, int64_t T, int64_t topk, int64_t E,
                                int32_t* offsets, int32_t* perm, int32_t* inv_perm,
                                unsigned* status, cudaStream_t st);
+// fp32 combine sums -> bf16 out, and the sums reset to zero.
+cudaError_t launch_moe_combine_finish(float* acc, int64_t T, int64_t N, int64_t ld_acc, void* out,
+                                      int64_t ldo, cudaStream_t st);
 cudaError_t launch_moe_combine(const void* y, int64_t ldy, const int32_t* inv_perm,
                                const float* w, int64_t T, int64_t topk, int64_t H, void* out,
                                int64_t ldo, cudaStream_t st);

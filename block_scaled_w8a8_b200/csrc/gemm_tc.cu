@@ -64,6 +64,8 @@ using tc::kMagicBits;
 using tc::TcParams;
 using tc::decode_tile;
 using tc::wrow_block;
+using tc::bf16_round;
+using tc::red_add_v4;
 using tc::make_tmap;
 using tc::sm_count;
 using tc::encode_fn;
@@ -281,6 +283,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int64_t n0 = (int64_t)nb * BN + CW * half;
       const float* sw_e = p.sw + (int64_t)e * p.sw_expert_stride;
       const int64_t swrow = n0 < p.N ? wrow_block(n0, p.seam, p.N) * p.Kb : 0;
+      // combine: this row's (token, slot) pair and routing weight, read
+      // before the K loop so their latency hides behind it
+      int pair = -1;
+      float comb_wt = 0.f;
+      if (p.comb_acc && row_ok) {
+        pair = __ldg(p.comb_perm + m);
+        if ((unsigned)pair < (unsigned)p.M) comb_wt = __ldg(p.comb_w + pair);
+      }
       float accf[CW];
 #pragma unroll
       for (int i = 0; i < CW; ++i) accf[i] = 0.f;
@@ -459,6 +469,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ++tcount;
         continue;
       }
+      if (p.comb_acc) {
+        // weighted top-k combine: add w[t, j] * bf16(y) to token t's fp32
+        // sums, each product rounded to fp32 once.  A sum starts from zero,
+        // so with top-2 (two terms) the atomic order cannot change it
+        if (row_ok && n0 < p.N) {
+          if ((unsigned)pair >= (unsigned)p.M) {
+            record_status(p.status, kStatusBadInput, 0x309u);
+          } else {
+            float* arow = p.comb_acc + (int64_t)(pair / p.topk) * p.ldo + n0;
+            if (n0 + CW <= p.N && ((reinterpret_cast<uintptr_t>(arow) & 15) == 0)) {
+#pragma unroll
+              for (int j = 0; j < CW; j += 4)
+                red_add_v4(arow + j, comb_wt * bf16_round(accf[j]),
+                           comb_wt * bf16_round(accf[j + 1]), comb_wt * bf16_round(accf[j + 2]),
+                           comb_wt * bf16_round(accf[j + 3]));
+            } else {
+              for (int j = 0; j < CW; ++j)
+                if (n0 + j < p.N) atomicAdd(arow + j, comb_wt * bf16_round(accf[j]));
+            }
+          }
+        }
+        continue;
+      }
       if (row_ok && n0 < p.N && p.out_f32) {
         float* frow = p.out_f32 + m * p.ldo + n0;
         if (n0 + CW <= p.N && ((reinterpret_cast<uintptr_t>(frow) & 15) == 0)) {
@@ -552,6 +585,7 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   p.status = a.status;
   p.q_out = static_cast<uint8_t*>(a.q_out); p.ldq = a.ldq; p.s_out = a.s_out;
   p.out_f32 = a.out_f32;
+  p.comb_acc = a.comb_acc; p.comb_perm = a.comb_perm; p.comb_w = a.comb_w; p.topk = (int)a.topk;
   const int64_t mblk_bound = (a.M + BM - 1) / BM + (a.offsets ? a.E : 0);
   const int64_t tiles_bound = mblk_bound * p.nblk;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles_bound, sm_count()));

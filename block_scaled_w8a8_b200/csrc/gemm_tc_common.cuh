@@ -34,7 +34,22 @@ struct TcParams {
   // [rows, I] (row stride ldq) and scales [I / 128][sa_rows] instead of out
   uint8_t* q_out; int64_t ldq; float* s_out;
   float* out_f32;                               // unrounded fp32 output (no bias) or null
+  // weighted top-k combine into fp32 token rows (w2 of the MoE layer) or null
+  float* comb_acc; const int32_t* comb_perm; const float* comb_w; int topk;
 };
+
+// Four fp32 atomic adds to consecutive, 16-byte aligned global addresses in
+// one vector reduction.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// x rounded to bf16 (nearest even) and back.
+__device__ __forceinline__ float bf16_round(float x) {
+  return bf16_bits_to_float(float_to_bf16_bits(x));
+}
 
 // Weight-scale row of output column n (block_n = 128).  A fused gate+up
 // weight blocks its halves separately: rows past the seam restart at

@@ -130,31 +130,6 @@ def router_logits(T: int, E: int, seed: int) -> torch.Tensor:
     return torch.randn(T, E, generator=g, dtype=torch.float32)
 
 
-def routing(T: int, E: int, topk: int, seed: int):
-    """Top-k routing from softmax of N(0,1) logits (harness choice).
-
-    Softmax in fp64; experts ranked by probability, ties to the lower index;
-    the top-k probabilities are renormalised to sum to one.  Returns
-    (ids int32 [T, topk], weights float32 [T, topk]) as numpy arrays."""
-    logits = router_logits(T, E, seed).double().numpy()
-    z = logits - logits.max(axis=1, keepdims=True)
-    p = np.exp(z)
-    p /= p.sum(axis=1, keepdims=True)
-    order = np.argsort(-p, axis=1, kind="stable")[:, :topk]
-    top = np.take_along_axis(p, order, axis=1)
-    w = top / top.sum(axis=1, keepdims=True)
-    return order.astype(np.int32), w.astype(np.float32)
-
-
-def moe_inputs(cfg: MoE, device="cpu"):
-    """(x bf16 [T, H], w13 fp32 [E, 2I, H], w2 fp32 [E, H, I], ids, topk_w)."""
-    x = activations(cfg.T, cfg.H, cfg.seed, 0, 1.0, device)
-    w13 = weights(2 * cfg.I, cfg.H, cfg.w_std, cfg.seed, device, batch=cfg.E)
-    w2 = weights(cfg.H, cfg.I, cfg.w_std, cfg.seed + 1, device, batch=cfg.E)
-    ids, tw = routing(cfg.T, cfg.E, cfg.topk, cfg.seed)
-    return x, w13, w2, ids, tw
-
-
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 bit patterns (CPU copy)."""
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)

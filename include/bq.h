@@ -367,6 +367,41 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
                                      int64_t block_k, int dtype, void* q, int64_t ldq, float* s,
                                      void* stream);
 
+/* The w2 grouped GEMM fused with the weighted top-k combine (block-wise INT8
+ * page, sections 5-6: the down projection, then each token's top-k expert
+ * outputs summed with their routing weights).  For each expert e and each
+ * row r in [expert_offsets[e], expert_offsets[e+1]), with p = perm[r] the
+ * row's (token, slot) pair t * topk + j:
+ *   y[r, :] = bf16(block-scaled GEMM of qa[r] against qw[e])  (as bq_grouped_gemm);
+ *   acc[t, :] += fp32(topk_w[p] * y[r, :])                      (fp32 atomic add).
+ * y is never stored.  acc: fp32 [T, N], T = R / topk (row stride ld_acc >= N;
+ * 16-byte aligned rows take vector atomics), must hold zeros on entry;
+ * bq_moe_combine_finish then rounds it once to bf16 and zeroes it again.
+ * Every sum starts from zero, so with topk <= 2 the atomic order cannot
+ * change it: out = bf16(fp32(w0*y0) + fp32(w1*y1)), deterministic.  With
+ * topk > 2 the fp32 sum's association follows the atomic order (each result
+ * is within the fp32 rounding of the sum, not bit-reproducible).
+ * qa: codes [R, K] (row stride lda), sa: fp32 [ceil(K/128)][R]; qw: codes
+ * [E, N, K] (dense), sw: fp32 [E][ceil(N/128)][ceil(K/128)]; perm: int32 [R]
+ * as bq_moe_permute writes it (an entry outside [0, R) is skipped and
+ * recorded in the device status word as BQ_ERR_INVALID_ARG); topk_w: fp32
+ * [T, topk].  Rows past expert_offsets[E] add nothing.  Needs R a multiple
+ * of topk, block_n = block_k = 128 (or block_k >= K) and the tensor-core
+ * path (BQ_PATH_AUTO, BQ_PATH_TCGEN05 or BQ_PATH_TCGEN05_1CTA); otherwise
+ * BQ_ERR_UNSUPPORTED.  Needs no workspace. */
+bq_status bq_grouped_gemm_combine(const void* qa, int64_t lda, const float* sa, int64_t R,
+                                  const int32_t* expert_offsets, int64_t E, const void* qw,
+                                  const float* sw, int64_t N, int64_t K, int64_t block_n,
+                                  int64_t block_k, int dtype, const int32_t* perm,
+                                  const float* topk_w, int64_t topk, float* acc, int64_t ld_acc,
+                                  void* stream);
+
+/* out[t, n] = bf16(acc[t, n]) (round to nearest even), then acc[t, n] = 0,
+ * for the fp32 sums bq_grouped_gemm_combine accumulated.  acc: fp32 [T, N]
+ * (row stride ld_acc >= N), out: bf16 [T, N] (row stride ldo >= N). */
+bq_status bq_moe_combine_finish(float* acc, int64_t T, int64_t N, int64_t ld_acc, void* out,
+                                int64_t ldo, void* stream);
+
 /* ---------------- MXFP8 dense linear ----------------
  * The SGLang quantization doc ("GEMM backends for FP4/FP8") lists an MXFP8
  * dense linear beside the blockwise FP8 GEMM but does not define the format;

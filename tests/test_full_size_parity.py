@@ -5,7 +5,9 @@ launch configuration that bench.py times:
   prefill up-proj INT8   M = 4096, N = 14336, K = 4096           (bq_quant_act + bq_gemm)
   blockwise FP8 linear   M = 2048, N = 4096,  K = 14336          (bq_quant_act + bq_gemm)
   MXFP8 linear           M = 2048, N = 4096,  K = 14336          (bq_mx_quant_act + bq_mx_gemm)
-  block-INT8 MoE layer   T = 4096, H = 4096, I = 14336, E = 8, top-2 (bench.MoeLayer)
+  block-INT8 MoE layer   T = 4096, H = 4096, I = 14336, E = 8, top-2 (bench.MoeLayer:
+                         device routing, the unfused stages, and the fused w13 and w2
+                         epilogues against them)
 
 Activation codes and scales are compared bit-exactly over the whole tensors;
 weight codes on whole 128-row block rows; GEMM outputs on sampled rows (every
@@ -141,9 +143,21 @@ def moe_layer():
     layer.run(bench.MoeLayer.UNFUSED)
     torch.cuda.synchronize()
     bq.check_device_status()
+    # the device routing's ids and weights, on the host, for the stages after it
+    layer.ids = layer.ids_d.cpu().numpy()
+    layer.tw = layer.tw_d.cpu().numpy()
     yield layer
     del layer
     torch.cuda.empty_cache()
+
+
+def test_moe_route_full_size(moe_layer):
+    """Device routing of the T x E logits: expert ids bit-exact, weights to
+    the fp32 rounding of the softmax (the oracle's is fp64)."""
+    L = moe_layer
+    ids, tw = oracle.moe_route(L.logits.cpu().numpy(), L.cfg.topk)
+    assert np.array_equal(L.ids, ids), "routed expert ids differ"
+    np.testing.assert_allclose(L.tw, tw, rtol=2e-6, atol=1e-7)
 
 
 def test_moe_permute_full_size(moe_layer):
@@ -248,6 +262,30 @@ def test_moe_combine_full_size(moe_layer):
     inv = L.inv.cpu().numpy()
     assert_combine_close(L.out, oracle.moe_combine(yb, inv, L.tw), yb, inv, L.tw)
     assert np.isfinite(bf16_values(L.out)).all()
+
+
+def test_moe_fused_w2_combine_full_size(moe_layer):
+    """The w2 GEMM with the combine in its epilogue (atomic fp32 sums, then
+    one bf16 rounding), on the full layer: against the oracle's combine of
+    the unfused w2 output (which test_moe_w2_sampled_rows pins), and, top-2
+    sums being order-free, bit-exact to the fp32 slot-order sum."""
+    L = moe_layer
+    c = L.cfg
+    acc = torch.zeros(c.T, c.H, dtype=torch.float32, device="cuda")
+    L.bq.grouped_gemm_combine(L.qh, L.sh, L.off, L.q2, L.s2, L.perm, L.tw_d, acc, c.dtype)
+    out = L.bq.moe_combine_finish(acc)
+    torch.cuda.synchronize()
+    L.bq.check_device_status()
+    yb = host_bits(L.y2)
+    inv = L.inv.cpu().numpy()
+    assert_combine_close(out, oracle.moe_combine(yb, inv, L.tw), yb, inv, L.tw, "fused combine")
+    yv = oracle.bf16_to_f64(yb).astype(np.float32)
+    s = np.zeros((c.T, c.H), np.float32)
+    for j in range(c.topk):
+        s = s + L.tw[:, j:j + 1] * yv[inv.reshape(c.T, c.topk)[:, j]]
+    exact = oracle.bf16_to_f64(oracle.bf16_from_f64(s.astype(np.float64)))
+    assert np.array_equal(bf16_values(out), exact), "atomic combine differs from the fp32 sum"
+    assert not acc.any(), "the finish pass must leave the sums zeroed"
 
 
 def test_moe_fused_w13_silu_requant_full_size(moe_layer):

@@ -351,7 +351,7 @@ def test_linear_tiny_workload(dtype):
 
 def moe_problem(T=200, H=256, I=192, E=8, topk=2, seed=21, dtype=INT8):
     x = act_bits(T, H, seed)
-    ids, tw = bq_synth.routing(T, E, topk, seed)
+    ids, tw = oracle.moe_route(bq_synth.router_logits(T, E, seed).numpy(), topk)
     w13 = bq_synth.weights(2 * I, H, 0.02, seed, batch=E).numpy()
     w2 = bq_synth.weights(H, I, 0.02, seed + 1, batch=E).numpy()
     q13, s13 = zip(*[oracle.quant_weight_gate_up(w13[e], I, 128, 128, dtype) for e in range(E)])
@@ -362,7 +362,7 @@ def moe_problem(T=200, H=256, I=192, E=8, topk=2, seed=21, dtype=INT8):
 
 def test_moe_permute_bit_exact():
     for T, E, topk in [(200, 8, 2), (1000, 8, 2), (37, 5, 3), (4096, 8, 2)]:
-        ids, _ = bq_synth.routing(T, E, topk, T)
+        ids, _ = oracle.moe_route(bq_synth.router_logits(T, E, T).numpy(), topk)
         off, perm, inv = bq.moe_permute(dev_i32(ids), E)
         o_ref, p_ref, i_ref = oracle.moe_permute(ids, E)
         assert np.array_equal(off.cpu().numpy(), o_ref)
@@ -439,6 +439,89 @@ def test_grouped_gemm_tcgen05_vs_oracle(path, dtype):
     ref13 = oracle.grouped_gemm(qx[rows], sx[rows], o_ref, p["q13"], p["s13"], 128, 128, dtype,
                                 seam=I)
     assert_gemm_close(y13, ref13, "tcgen05 grouped w13")
+
+
+# w2 grouped GEMM fused with the weighted top-k combine
+# (T, H, I, E, topk, dtype, seed): two 256-wide column tiles, FP8, an output
+# width with a ragged last tile (scalar atomics), top-3 (order-dependent fp32
+# sums: tolerance only), top-1, and K with a partial last block
+COMBINE_CASES = [(300, 384, 256, 8, 2, INT8, 41), (300, 384, 256, 8, 2, FP8, 42),
+                 (200, 208, 256, 5, 2, INT8, 43), (100, 256, 128, 4, 3, INT8, 44),
+                 (64, 256, 256, 4, 1, FP8, 45), (150, 512, 320, 8, 2, INT8, 46)]
+
+
+def _combine_exact(y_bits, inv, w):
+    """bf16 of the fp32 sum of fp32 products w[t, j] * y[inv[t, j]], summed in
+    slot order from zero: what the atomic combine computes for top-k <= 2."""
+    T, topk = w.shape
+    yv = oracle.bf16_to_f64(y_bits).astype(np.float32)
+    acc = np.zeros((T, y_bits.shape[1]), np.float32)
+    for j in range(topk):
+        acc = acc + w[:, j:j + 1] * yv[inv.reshape(T, topk)[:, j]]
+    return oracle.bf16_to_f64(oracle.bf16_from_f64(acc.astype(np.float64)))
+
+
+@pytest.mark.parametrize("T,H,I,E,topk,dtype,seed", COMBINE_CASES)
+def test_grouped_gemm_combine_vs_oracle(T, H, I, E, topk, dtype, seed):
+    p = moe_problem(T=T, H=H, I=I, E=E, topk=topk, dtype=dtype, seed=seed)
+    off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), E)
+    o_ref, p_ref, i_ref = oracle.moe_permute(p["ids"], E)
+    qa, sa = bq.moe_quant_gather(dev_bf16(p["x"]), perm, topk, 128, dtype)
+    if I % 128 == 0:
+        qh, sh = bq.grouped_gemm_silu_quant(qa, sa, off, dev_u8(p["q13"]), dev_f32(p["s13"]),
+                                            dtype)
+    else:   # the fused SiLU epilogue needs whole 128-column h groups
+        y13 = bq.grouped_gemm(qa, sa, off, dev_u8(p["q13"]), dev_f32(p["s13"]), 128, 128,
+                              n_seam=I, dtype=dtype)
+        qh, sh = bq.moe_silu_mul_quant(y13, I, 128, dtype)
+    q2, s2, tw = dev_u8(p["q2"]), dev_f32(p["s2"]), dev_f32(p["tw"])
+    # the unfused w2 GEMM on the same tensor-core kernel: its bf16 rows are the
+    # y the combining epilogue weights, and they are pinned to the oracle
+    bq.set_path(bq.PATH_TCGEN05_1CTA)
+    y2 = bq.grouped_gemm(qh, sh, off, q2, s2, 128, 128, 0, dtype)
+    acc = torch.zeros(T, H, dtype=torch.float32, device="cuda")
+    bq.grouped_gemm_combine(qh, sh, off, q2, s2, perm, tw, acc, dtype)
+    out = bq.moe_combine_finish(acc)
+    torch.cuda.synchronize()
+    bq.check_device_status()
+    ref2 = oracle.grouped_gemm(qh.cpu().numpy(), sh.cpu().numpy().T,
+                               o_ref, p["q2"], p["s2"], 128, 128, dtype)
+    assert_gemm_close(y2, ref2, "w2")
+    yb = host_bits(y2)
+    assert_combine_close(out, oracle.moe_combine(yb, i_ref, p["tw"]), yb, i_ref, p["tw"],
+                         "fused combine")
+    if topk <= 2:
+        g = bf16_values(out)
+        assert np.array_equal(g, _combine_exact(yb, i_ref, p["tw"])), \
+            "atomic combine differs from the fp32 slot-order sum"
+    assert not acc.any(), "the finish pass must leave the sums zeroed"
+    # a second layer call on the zeroed sums gives the same bits
+    bq.grouped_gemm_combine(qh, sh, off, q2, s2, perm, tw, acc, dtype)
+    out2 = bq.moe_combine_finish(acc)
+    torch.cuda.synchronize()
+    if topk <= 2:
+        assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+
+
+def test_grouped_gemm_combine_reports_a_bad_pair_index():
+    p = moe_problem(T=64, H=256, I=128, E=4, topk=2, seed=47)
+    off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), 4)
+    qa, sa = bq.moe_quant_gather(dev_bf16(p["x"]), perm, 2, 128, INT8)
+    qh, sh = bq.grouped_gemm_silu_quant(qa, sa, off, dev_u8(p["q13"]), dev_f32(p["s13"]), INT8)
+    bad = perm.clone()
+    bad[5] = 128                                   # outside [0, R): skipped and recorded
+    acc = torch.zeros(64, 256, dtype=torch.float32, device="cuda")
+    bq.grouped_gemm_combine(qh, sh, off, dev_u8(p["q2"]), dev_f32(p["s2"]), bad,
+                            dev_f32(p["tw"]), acc, INT8)
+    torch.cuda.synchronize()
+    with pytest.raises(bq.BqError) as ei:
+        bq.check_device_status()
+    assert ei.value.status == bq.ERR_INVALID_ARG
+    bq.check_device_status()                       # read and cleared
+    with pytest.raises(bq.BqError) as ei:
+        bq.grouped_gemm_combine(qh[:127], sh[:, :127].contiguous(), off, dev_u8(p["q2"]),
+                                dev_f32(p["s2"]), perm[:127], dev_f32(p["tw"]), acc, INT8)
+    assert ei.value.status == bq.ERR_INVALID_ARG   # R is not T * topk
 
 
 # w13 grouped GEMM fused with silu(gate) * up and the 1 x 128 requantisation

@@ -379,7 +379,7 @@ def test_quantised_linear_close_to_dense():
 # --------------------------------------------------------------------------
 
 def test_moe_permute_matches_stable_sort():
-    ids, _ = bq_synth.routing(500, 8, 2, 3)
+    ids, _ = oracle.moe_route(bq_synth.router_logits(500, 8, 3).numpy(), 2)
     off, perm, inv = oracle.moe_permute(ids, 8)
     flat = ids.reshape(-1)
     assert off[-1] == flat.size
@@ -409,7 +409,7 @@ def test_combine_identity_experts():
     # permute, identity experts (y = gathered x), weights 1/topk: combine == x
     T, H, topk = 33, 24, 2
     x = _random_bf16((T, H), 14)
-    ids, _ = bq_synth.routing(T, 8, topk, 4)
+    ids, _ = oracle.moe_route(bq_synth.router_logits(T, 8, 4).numpy(), topk)
     off, perm, inv = oracle.moe_permute(ids, 8)
     y = x[perm // topk]
     w = np.full((T, topk), 1.0 / topk, np.float32)

@@ -130,7 +130,7 @@ def _worker(rank, world, port, case, q):
         elif case == "moe":
             T, H, I, E, topk = 24, 256, 256, 4, 2
             x = bq_synth.activations(T, H, 10 + rank)      # each rank's own tokens
-            ids, tw = bq_synth.routing(T, E, topk, 20 + rank)
+            ids, tw = oracle.moe_route(bq_synth.router_logits(T, E, 20 + rank).numpy(), topk)
             w13 = [bq_synth.weights(2 * I, H, 0.02, 30 + e).numpy() for e in range(E)]
             w2 = [bq_synth.weights(H, I, 0.02, 40 + e).numpy() for e in range(E)]
             qs13 = [oracle.quant_weight_gate_up(w, I, 128, 128, oracle.INT8) for w in w13]

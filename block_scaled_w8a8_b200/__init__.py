@@ -22,7 +22,8 @@ import torch
 INT8 = 0
 FP8_E4M3 = 1
 
-PATH_AUTO, PATH_SIMT, PATH_TCGEN05, PATH_DECODE, PATH_TCGEN05_1CTA = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_SIMT, PATH_TCGEN05, PATH_DECODE, PATH_TCGEN05_1CTA, PATH_TCGEN05_PAIR = \
+    0, 1, 2, 3, 4, 5
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT = range(7)

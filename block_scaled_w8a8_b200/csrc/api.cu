@@ -99,8 +99,18 @@ const char* bq_status_string(int s) {
 
 const char* bq_last_error_message(void) { return g_msg; }
 
+// Paths that run the tensor-core kernels; the tile shape a forced path picks.
+static bool tc_path(int path) {
+  return path == BQ_PATH_AUTO || path == BQ_PATH_TCGEN05 || path == BQ_PATH_TCGEN05_1CTA ||
+         path == BQ_PATH_TCGEN05_PAIR;
+}
+
+static int tc_shape(int path) {
+  return path == BQ_PATH_TCGEN05_1CTA ? 1 : path == BQ_PATH_TCGEN05_PAIR ? 2 : 0;
+}
+
 bq_status bq_set_path(int path) {
-  BQ_CHECK_ARG(path >= BQ_PATH_AUTO && path <= BQ_PATH_TCGEN05_1CTA, "unknown path %d", path);
+  BQ_CHECK_ARG(path >= BQ_PATH_AUTO && path <= BQ_PATH_TCGEN05_PAIR, "unknown path %d", path);
   g_path = path;
   return ok();
 }
@@ -528,7 +538,7 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
   if (R == 0 || I == 0) return ok();
   BQ_CHECK_ARG(q && s && expert_offsets, "q, s and expert_offsets must not be NULL");
   BQ_CHECK_ARG(K == 0 || (qa && sa && qw13 && sw13), "qa, sa, qw13 and sw13 must not be NULL");
-  if (!(g_path == BQ_PATH_AUTO || g_path == BQ_PATH_TCGEN05 || g_path == BQ_PATH_TCGEN05_1CTA))
+  if (!tc_path(g_path))
     return fail(BQ_ERR_UNSUPPORTED, "the fused SiLU GEMM runs on the tensor-core path only");
   const int64_t Kb = cdiv(K, block_k);
   bq::GemmArgs a{};
@@ -540,6 +550,7 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
   a.offsets = expert_offsets; a.E = E;
   a.w_expert_stride = 2 * I * K; a.sw_expert_stride = a.Nbs * Kb;
   a.q_out = q; a.ldq = ldq; a.s_out = s;
+  a.tc_shape = tc_shape(g_path);
   char why[256] = "";
   if (!bq::tc_silu_supported(a, why, sizeof(why))) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
   unsigned* w = nullptr;
@@ -566,7 +577,7 @@ bq_status bq_grouped_gemm_combine(const void* qa, int64_t lda, const float* sa, 
   BQ_CHECK_ARG(acc && perm && topk_w && expert_offsets,
                "acc, perm, topk_w and expert_offsets must not be NULL");
   BQ_CHECK_ARG(K == 0 || (qa && sa && qw && sw), "qa, sa, qw and sw must not be NULL");
-  if (!(g_path == BQ_PATH_AUTO || g_path == BQ_PATH_TCGEN05 || g_path == BQ_PATH_TCGEN05_1CTA))
+  if (!tc_path(g_path))
     return fail(BQ_ERR_UNSUPPORTED, "the combining GEMM runs on the tensor-core path only");
   const int64_t Kb = cdiv(K, block_k);
   bq::GemmArgs a{};
@@ -578,6 +589,7 @@ bq_status bq_grouped_gemm_combine(const void* qa, int64_t lda, const float* sa, 
   a.offsets = expert_offsets; a.E = E;
   a.w_expert_stride = N * K; a.sw_expert_stride = a.Nbs * Kb;
   a.comb_acc = acc; a.comb_perm = perm; a.comb_w = topk_w; a.topk = topk;
+  a.tc_shape = tc_shape(g_path);
   char why[256] = "";
   if (!bq::tc_supported(a, why, sizeof(why))) return fail(BQ_ERR_UNSUPPORTED, "%s", why);
   unsigned* w = nullptr;
@@ -650,7 +662,7 @@ bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* q
     return fail(BQ_ERR_UNSUPPORTED, "MXFP8 GEMM needs K a positive multiple of 128");
   if (M == 0 || N == 0) return ok();
   BQ_CHECK_ARG(qa && sfa && qw && sfw && out, "qa, sfa, qw, sfw and out must not be NULL");
-  if (!(g_path == BQ_PATH_AUTO || g_path == BQ_PATH_TCGEN05 || g_path == BQ_PATH_TCGEN05_1CTA))
+  if (!tc_path(g_path))
     return fail(BQ_ERR_UNSUPPORTED, "the MXFP8 GEMM runs on the tensor-core path only");
   if (lda % 16 != 0 || ldw % 16 != 0 || !aligned16(qa) || !aligned16(qw) || !aligned16(sfa) ||
       !aligned16(sfw))

@@ -51,6 +51,8 @@ struct GemmArgs {
   // and bias are unused and row m adds comb_w[comb_perm[m]] * bf16(row m) to
   // fp32 row comb_perm[m] / topk of comb_acc (row stride ldo) atomically
   float* comb_acc; const int32_t* comb_perm; const float* comb_w; int64_t topk;
+  // tcgen05 tile shape: 0 chosen by size, 1 one CTA per tile, 2 CTA pairs
+  int tc_shape;
 };
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t st);

@@ -38,7 +38,9 @@ static int run_simt(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
   return kRunOk;
 }
 
-static int run_tc(const GemmArgs& a, cudaStream_t st, char* why, size_t n) {
+static int run_tc(const GemmArgs& a0, int path, cudaStream_t st, char* why, size_t n) {
+  GemmArgs a = a0;
+  a.tc_shape = path == BQ_PATH_TCGEN05_1CTA ? 1 : path == BQ_PATH_TCGEN05_PAIR ? 2 : 0;
   cudaError_t e = launch_gemm_tc(a, st);
   if (e != cudaSuccess) {
     snprintf(why, n, "tcgen05 GEMM launch: %s", cudaGetErrorString(e));
@@ -94,7 +96,7 @@ static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes
         return run_cluster_decode(d, st, why, why_len);
       if (a.M <= kDecodeMaxRows && !a.out_f32 && decode_supported(a, nullptr, 0))
         return run_decode(a, ws, ws_bytes, pdl, st, why, why_len);
-      if (a.M > kDecodeMaxRows && tc_supported(a, nullptr, 0)) return run_tc(a, st, why, why_len);
+      if (a.M > kDecodeMaxRows && tc_supported(a, nullptr, 0)) return run_tc(a, path, st, why, why_len);
       return run_simt(a, st, why, why_len);
     }
     case BQ_PATH_DECODE: {
@@ -112,8 +114,9 @@ static int dispatch_dense(const GemmArgs& a, int path, void* ws, size_t ws_bytes
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
     case BQ_PATH_TCGEN05_1CTA:
+    case BQ_PATH_TCGEN05_PAIR:
       if (!tc_supported(a, why, why_len)) return kRunUnsupported;
-      return run_tc(a, st, why, why_len);
+      return run_tc(a, path, st, why, why_len);
     default:
       snprintf(why, why_len, "kernel path %d is not available in this build", path);
       return kRunUnsupported;
@@ -136,14 +139,15 @@ int run_grouped_gemm(const GemmArgs& a, int path, void* ws, size_t ws_bytes, cud
   (void)ws_bytes;
   switch (path) {
     case BQ_PATH_AUTO:
-      if (tc_supported(a, nullptr, 0)) return run_tc(a, st, why, why_len);
+      if (tc_supported(a, nullptr, 0)) return run_tc(a, path, st, why, why_len);
       return run_simt(a, st, why, why_len);
     case BQ_PATH_SIMT:
       return run_simt(a, st, why, why_len);
     case BQ_PATH_TCGEN05:
     case BQ_PATH_TCGEN05_1CTA:
+    case BQ_PATH_TCGEN05_PAIR:
       if (!tc_supported(a, why, why_len)) return kRunUnsupported;
-      return run_tc(a, st, why, why_len);
+      return run_tc(a, path, st, why, why_len);
     default:
       snprintf(why, why_len, "kernel path %d is not available for grouped GEMM", path);
       return kRunUnsupported;

@@ -4,32 +4,33 @@
 // (block-wise INT8 page, sections 2 and 4; blockwise FP8 of the SGLang
 // quantization doc, "GEMM backends for FP4/FP8"), for block_n = block_k = 128.
 //
-// Design (persistent, warp-specialised, one CTA per SM):
-//   warps 0, 2  TMA producers: per K-block, warp 0 loads one 128x128 A tile
-//               and warp 2 one BNx128 W tile (BN = 256, or 128 for narrow
-//               problems; K-major, 128-byte swizzle) into
-//               an S-stage ring (one issuing thread alone cannot sustain the
-//               L2->SMEM rate a K-block needs).
-//   warp 1      MMA issuer (lane 0): 4 x tcgen05.mma (K = 32 each) per K-block
-//               into a TMEM buffer; the buffer holds exactly one K-block's
-//               partial P_kb (int32 for kind::i8, fp32 for kind::f8f6f4).
-//               512 / BN TMEM buffers (all 512 columns) rotate, so the MMA
-//               runs ahead of the promotion and the TMEM hand-off latency
-//               stays off the critical path.  Also owns the TMEM allocation.
+// Design (persistent, warp-specialised, one CTA per SM or one CTA pair per
+// two SMs):
+//   warps 0, 2, 3  TMA producers: K-block j of the CTA's sequence goes to
+//               producer j % 3, which loads its 128x128 A tile and its W
+//               tile (BN x 128, or BN/2 x 128 per CTA of a pair; K-major,
+//               128-byte swizzle) into an S-stage ring.  One issuing thread
+//               sustains about one TMA tile per 270 ns on B200.
+//   warp 1      MMA issuer (lane 0 alone): 4 x tcgen05.mma (K = 32 each) per
+//               K-block into a TMEM buffer; the buffer holds exactly one
+//               K-block's partial P_kb (int32 for kind::i8, fp32 for
+//               kind::f8f6f4).  512 / BN TMEM buffers (all 512 columns)
+//               rotate.  Also owns the TMEM allocation.
 //   warps 4-19  epilogue: warp w reads TMEM lanes 32*(w%4).. (one output row
 //               per thread) and columns [BN/4*h, BN/4*(h+1)), h = (w-4)/4; it
 //               promotes acc += P_kb * (sa[kb][m] * sw[nb][kb]) in fp32
 //               registers (scalar FADD/FFMA: measured faster here than the
-//               packed f32x2 forms), frees the buffer, and
-//               after the last K-block adds the bias and stores bf16.
+//               packed f32x2 forms), frees the buffer, and after the last
+//               K-block adds the bias and stores bf16 with 32-byte stores.
 //   registers   setmaxnreg moves registers from the control warpgroup (56
 //               each) to the epilogue (104 each): no spills in the
 //               promotion loop (+5% INT8, +3% FP8 measured).
-// INT8 promotion without the int->float conversion unit: since
-// |P_kb| <= 128 * 128 * 128 < 2^22, the integer sum P_kb + 0x4B400000 (an
-// integer add) has the bits of the float 12582912 + P_kb
-// exactly, so one FADD recovers P_kb exactly and one FFMA promotes it (FMA
-// pipe).
+// INT8 promotion without an integer add or the int->float conversion unit:
+// each TMEM buffer is pre-filled with the bits 0x4B400000 (the float
+// 1.5 * 2^23), so the MMA's int32 sum 0x4B400000 + P_kb (|P_kb| <=
+// 128 * 127 * 127 < 2^22) is the float 12582912 + P_kb exactly; one FADD
+// recovers P_kb exactly and one FFMA promotes it.  The epilogue refills
+// the buffer (tcgen05.st) as it frees it.
 // A tile scheduler walks (expert, m-block, n-block) tiles; a dense problem is
 // one expert.  The grouped (MoE) problem reads its expert row ranges from
 // device memory, so no host read-back is needed.  Rows of a tile past the
@@ -84,10 +85,15 @@ static_assert(kSplitRegs <= 65536, "register split exceeds the SM's register fil
 // TMEM accumulators of BN columns: all 512 columns (4 x 128 or 2 x 256)
 template <int BN>
 constexpr int tbufs() { return 512 / BN; }
+// TMA producer warps (0, 2 and 3), each issuing whole K-blocks in turn
+constexpr int kProducers = 3;
 
-template <int BN, int S>
+// Per CTA: an S-stage ring of one 128-row A tile and the CTA's W rows (all
+// BN of them, or BN / 2 for a CTA pair, which splits the MMA's N between its
+// two CTAs' shared memory).
+template <int BN, int S, bool PAIR = false>
 struct Smem {
-  static constexpr uint32_t kA = BM * BK, kB = BN * BK;
+  static constexpr uint32_t kA = BM * BK, kB = (PAIR ? BN / 2 : BN) * BK;
   static constexpr uint32_t kStages = S * (kA + kB);
   static constexpr uint32_t kBars = (2 * S + 2 * tbufs<BN>() + 6) * 8;
   static constexpr uint32_t kMisc = 8 + 2 * (kMaxE + 1) * 4;
@@ -100,12 +106,32 @@ struct Smem {
 // activation scales, per-channel or per-row-block weight scales).  The MMAs
 // then accumulate a tile's whole K in TMEM and the epilogue promotes once per
 // tile, out = P * sa[m] * sw[n / block_n], instead of once per K-block.
-template <int DT, int BN, int S, bool ONEK, bool SILU>
+//
+// PAIR: a cluster of two CTAs on two SMs computes a 256 x BN tile with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages its own 128 rows of A
+// and BN / 2 rows of W per K-block (the MMA reads the other half of W from
+// the peer's shared memory), so a K-block moves half the W bytes per SM of
+// the single-CTA kernel: L2 -> shared memory traffic per output falls by a
+// third at BN = 256.  Each CTA's TMEM receives its own 128 rows of the
+// accumulator, so the epilogue is the single-CTA one.  The leader (cluster
+// rank 0) issues the MMAs; loads of both CTAs complete on the leader's stage
+// barriers (cta_group::2 loads, no multicast); MMA completions are committed
+// to both CTAs' barriers; both CTAs' epilogues release a TMEM buffer on the
+// leader's barrier.
+template <int DT, int BN, int S, bool ONEK, bool SILU, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcParams p) {
-  using L = Smem<BN, S>;
+  using L = Smem<BN, S, PAIR>;
   constexpr int kTBufs = tbufs<BN>();
+  constexpr int TM = PAIR ? 2 * BM : BM;           // rows of a scheduled tile
+  constexpr int BNL = PAIR ? BN / 2 : BN;          // W rows this CTA stages
+  // INT8 K-block partials land on a TMEM buffer pre-filled with the bits of
+  // 1.5 * 2^23: the int32 sum 0x4B400000 + P_kb is then the float
+  // 12582912 + P_kb exactly (|P_kb| <= 128 * 127 * 127 < 2^22), so the
+  // epilogue needs one FADD and one FFMA per element and no integer add; it
+  // refills the buffer with the bias as it frees it
+  constexpr bool kBias = DT == kInt8 && !ONEK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,80 +156,104 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 2);            // the A producer and the B producer
+      mbar_init(smem_u32(&full[s]), 1);            // the (leader's) producer of the K-block
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < kTBufs; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), kEpiWarps);
+      mbar_init(smem_u32(&tempty[b]), (PAIR ? 2 : 1) * kEpiWarps);   // (leader's) epilogues
     }
     mbar_init(smem_u32(&drain[0]), 1);
     for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&xbar[i]), kEpiWarps / 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmA);
-  if (warp == 2 && lane == 0) tma_prefetch_desc(&tmB);
+  if (warp != 1 && warp < 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
   // expert row ranges (sanitised: clamped to [0, M] and nondecreasing)
-  if (threadIdx.x == 32) tc::load_expert_ranges<BM>(p, off_s, tp_s);
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTBufs * BN);
+  if (threadIdx.x == 32) tc::load_expert_ranges<TM>(p, off_s, tp_s);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_alloc_pair(smem_u32(tmem_slot), kTBufs * BN);
+    else tmem_alloc(smem_u32(tmem_slot), kTBufs * BN);
+  }
   tc_fence_before();
-  __syncthreads();
+  // a pair's barriers all exist before any load, commit or arrive signals them
+  if constexpr (PAIR) cluster_sync_all();
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tp_s[E];
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;      // 0: the pair's leader
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (warp < 4) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kCtrlRegs) : "memory");
-  if (warp == 0 || warp == 2) {
-    // ---------------- TMA producers: warp 0 the A tiles, warp 2 the W tiles
-    // (one issuing thread sustains only part of the L2->SMEM rate a K-block
-    // needs; two issue in parallel) ----------------
-    const bool is_a = warp == 0;
-    int stage = 0;
+  if (warp != 1) {
+    // ---------------- TMA producers: warps 0, 2 and 3 take whole K-blocks
+    // in turn (K-block j of this CTA's sequence goes to producer j % 3), each
+    // issuing the A tile and the W tile of its K-blocks.  An issuing thread
+    // sustains about one TMA tile per 270 ns on B200, whatever the tile's
+    // size, so three issuers keep a 128 x 256 K-block's two tiles ahead of
+    // the tensor pipe ----------------
+    const int me = warp == 0 ? 0 : warp - 1;            // 0, 1, 2
+    // the leader's stage barriers in the cluster window
+    const uint32_t full_c0 = PAIR ? mapa_shared(smem_u32(&full[0]), 0) : smem_u32(&full[0]);
+    int stage = 0, j = 0;
     uint32_t phase = 0;
     int issued_parity[S];
 #pragma unroll
     for (int s = 0; s < S; ++s) issued_parity[s] = -1;
     int e_hint = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = unit0; t < total && ok; t += nunits) {
       int e, mb, nb;
-      decode_tile<BM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
-      const int a_row = off_s[e] + mb * BM;
-      const int b_row = e * (int)p.N + nb * BN;
-      for (int kb = 0; kb < p.Kmma; ++kb) {
-        if (!warp_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.status, 0x301u)) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          if (is_a) {
-            mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kA);
-            tma_load_2d(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, smem_u32(&full[stage]));
-          } else if (SILU) {
-            // 128 gate rows, then the 128 up rows of the same h columns: the
-            // MMA's N = 256 operand is the two boxes back to back
-            mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kB);
-            const int g_row = e * (int)p.N + nb * 128;
-            tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, g_row,
-                        smem_u32(&full[stage]));
-            tma_load_2d(smem_u32(sB + stage * L::kB + 128 * BK), &tmB, kb * BK,
-                        g_row + (int)p.seam, smem_u32(&full[stage]));
-          } else {
-            mbar_arrive_expect_tx(smem_u32(&full[stage]), L::kB);
-            tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, b_row, smem_u32(&full[stage]));
+      decode_tile<TM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
+      const int a_row = off_s[e] + mb * TM + BM * (int)rank;
+      const int b_row = e * (int)p.N + nb * BN + BNL * (int)rank;
+      for (int kb = 0; kb < p.Kmma; ++kb, ++j) {
+        if (j % kProducers == me) {
+          if (!warp_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.status, 0x301u)) {
+            ok = false;
+            break;
           }
+          if (PAIR && lane == 0) {
+            // the leader's barrier counts the bytes of both CTAs' loads
+            const uint32_t bar = full_c0 + 8u * (uint32_t)stage;
+            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (L::kA + L::kB));
+            tma_load_2d_pair(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, bar);
+            // SILU: the leader stages the 128 gate rows of the h columns, the
+            // peer the 128 up rows, so the MMA's N = 256 operand is gate | up
+            const int w_row = SILU ? e * (int)p.N + nb * 128 + (int)rank * (int)p.seam : b_row;
+            tma_load_2d_pair(smem_u32(sB + stage * L::kB), &tmB, kb * BK, w_row, bar);
+          } else if (lane == 0) {
+            const uint32_t bar = smem_u32(&full[stage]);
+            mbar_arrive_expect_tx(bar, L::kA + L::kB);
+            tma_load_2d(smem_u32(sA + stage * L::kA), &tmA, kb * BK, a_row, bar);
+            if (SILU) {
+              // 128 gate rows, then the 128 up rows of the same h columns:
+              // the MMA's N = 256 operand is the two boxes back to back
+              const int g_row = e * (int)p.N + nb * 128;
+              tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, g_row, bar);
+              tma_load_2d(smem_u32(sB + stage * L::kB + 128 * BK), &tmB, kb * BK,
+                          g_row + (int)p.seam, bar);
+            } else {
+              tma_load_2d(smem_u32(sB + stage * L::kB), &tmB, kb * BK, b_row, bar);
+            }
+          }
+          issued_parity[stage] = (int)phase;
         }
-        issued_parity[stage] = (int)phase;
         if (++stage == S) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
-    if (!ok) {
-      // drain: wait (bounded) for every load this warp issued
+    if (!ok && rank == 0) {
+      // drain: wait (bounded) for every load this warp issued (a pair's
+      // loads, the peer's too, complete on the leader's barriers)
       for (int s = 0; s < S; ++s) {
         if (issued_parity[s] < 0) continue;
         const uint64_t t0 = globaltimer();
@@ -213,53 +263,66 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    constexpr uint32_t idesc = instr_desc<DT>(BM, BN);
-    int stage = 0;
-    uint32_t phase = 0, kcount = 0;
-    int e_hint = 0;
-    bool ok = true, issued_any = false;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      for (int kb = 0; kb < p.Kmma; ++kb) {
-        // a TMEM buffer holds one K-block's partial, or (ONEK) a whole tile's
-        const bool unit_first = !ONEK || kb == 0;
-        const bool unit_last = !ONEK || kb == p.Kmma - 1;
-        const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
-        if ((unit_first && !warp_wait(smem_u32(&tempty[buf]), (tround & 1) ^ 1, abort_flag,
-                                      p.status, 0x302u)) ||
-            !warp_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x303u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
+    // ---------------- MMA issuer: lane 0 of warp 1 (of a pair's leader) ----
+    // One thread, no warp-wide waits or syncs per K-block: the tensor pipe
+    // queues little more than one K-block of MMAs, so any per-iteration
+    // overhead in the issuing loop shows up as idle tensor cycles.
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = instr_desc<DT>(TM, BN);
+      int stage = 0;
+      uint32_t phase = 0, kcount = 0;
+      bool ok = true, issued_any = false;
+      for (int t = unit0; t < total && ok; t += nunits) {
+        for (int kb = 0; kb < p.Kmma; ++kb) {
+          // a TMEM buffer holds one K-block's partial, or (ONEK) a whole tile's
+          const bool unit_first = !ONEK || kb == 0;
+          const bool unit_last = !ONEK || kb == p.Kmma - 1;
+          const uint32_t buf = kcount % kTBufs, tround = kcount / kTBufs;
+          // a biased buffer's first release is the epilogue's initial fill
+          const uint32_t tpar = kBias ? (tround & 1) : ((tround & 1) ^ 1);
+          if ((unit_first && !mbar_wait(smem_u32(&tempty[buf]), tpar, abort_flag, p.status,
+                                        0x302u)) ||
+              !mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.status, 0x303u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const uint32_t d = tmem_base + buf * BN;
           const uint64_t a0 = smem_desc_k128(smem_u32(sA + stage * L::kA));
           const uint64_t b0 = smem_desc_k128(smem_u32(sB + stage * L::kB));
+          if constexpr (PAIR) {
 #pragma unroll
-          for (int j = 0; j < BK / 32; ++j)
-            mma<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc,
-                    (j > 0 || !unit_first) ? 1u : 0u);
-          mma_commit(smem_u32(&empty[stage]));
-          if (unit_last) mma_commit(smem_u32(&tfull[buf]));
+            for (int j = 0; j < BK / 32; ++j)
+              mma_pair<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc,
+                           (kBias || j > 0 || !unit_first) ? 1u : 0u);
+            mma_commit_pair(smem_u32(&empty[stage]), (uint16_t)0x3);
+            if (unit_last) mma_commit_pair(smem_u32(&tfull[buf]), (uint16_t)0x3);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BK / 32; ++j)
+              mma<DT>(d, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(2 * j), idesc,
+                      (kBias || j > 0 || !unit_first) ? 1u : 0u);
+            mma_commit(smem_u32(&empty[stage]));
+            if (unit_last) mma_commit(smem_u32(&tfull[buf]));
+          }
+          issued_any = true;
+          if (unit_last) ++kcount;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
-        __syncwarp();
-        issued_any = true;
-        if (unit_last) ++kcount;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
+      }
+      if (!ok && issued_any) {
+        // wait (bounded) for the issued MMAs before the teardown frees TMEM
+        if constexpr (PAIR) mma_commit_pair(smem_u32(&drain[0]), (uint16_t)0x1);
+        else mma_commit(smem_u32(&drain[0]));
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(&drain[0]), 0) && globaltimer() - t0 < 100000000ull) {
         }
       }
     }
-    (void)e_hint;
-    if (!ok && issued_any) {
-      if (lane == 0) mma_commit(smem_u32(&drain[0]));
-      __syncwarp();
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(smem_u32(&drain[0]), 0) && globaltimer() - t0 < 100000000ull) {
-      }
-    }
+    __syncwarp();
   }
   } else {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kEpiRegs) : "memory");
@@ -271,13 +334,43 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int rit = 32 * q + lane;                 // row inside the tile
     const uint32_t tcol = (uint32_t)(CW * half);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // hand a TMEM buffer back to the MMA: the leader's barrier (a pair's
+    // peer arrives on it remotely)
+    const uint32_t tempty_c0 = PAIR ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
+    auto release_tmem = [=](uint32_t buf) {
+      if (PAIR && rank != 0) mbar_arrive_remote(tempty_c0 + 8u * buf);
+      else mbar_arrive(smem_u32(&tempty[buf]));
+    };
+    // this warp's TMEM columns of a buffer: CW from tcol, or (SILU) the 32
+    // gate and the 32 up columns of its h columns
+    auto fill_bias = [=](uint32_t buf) {
+      const uint32_t b0 = tmem_base + lane_base + buf * BN;
+      if constexpr (SILU) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          tmem_st4_fill(b0 + 32u * (uint32_t)half + 4u * j, kMagicBits);
+          tmem_st4_fill(b0 + 128u + 32u * (uint32_t)half + 4u * j, kMagicBits);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < CW / 4; ++j) tmem_st4_fill(b0 + tcol + 4u * j, kMagicBits);
+      }
+    };
+    if constexpr (kBias) {
+      for (int b = 0; b < kTBufs; ++b) fill_bias((uint32_t)b);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        for (int b = 0; b < kTBufs; ++b) release_tmem((uint32_t)b);
+    }
     uint32_t kcount = 0, tcount = 0;
     int e_hint = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = unit0; t < total && ok; t += nunits) {
       int e, mb, nb;
-      decode_tile<BM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
-      const int row0 = off_s[e] + mb * BM;
+      decode_tile<TM>(t, tp_s, off_s, E, e_hint, e, mb, nb);
+      const int row0 = off_s[e] + mb * TM + BM * (int)rank;
       const int64_t m = (int64_t)row0 + rit;
       const bool row_ok = rit < off_s[e + 1] - row0;
       const int64_t n0 = (int64_t)nb * BN + CW * half;
@@ -316,7 +409,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (c == CW / RC - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
+            if (lane == 0) release_tmem(buf);   // TMEM free for the MMA
           }
 #pragma unroll
           for (int i = 0; i < RC; ++i) {
@@ -353,18 +446,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t r[16];
             tmem_ld16(tb + (c < 2 ? 16u * c : 128u + 16u * (c - 2)), r);
             tmem_ld_wait();
-            if (c == 3) {
+            if (!kBias && c == 3) {
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
+              if (lane == 0) release_tmem(buf);   // TMEM free for the MMA
             }
             const float f = c < 2 ? fg : fu;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float x = DT == kInt8 ? __uint_as_float(r[i] + kMagicBits) - kMagic
-                                          : __uint_as_float(r[i]);
+              const float x = kBias ? __uint_as_float(r[i]) - kMagic : __uint_as_float(r[i]);
               accf[16 * c + i] = fmaf(x, f, accf[16 * c + i]);
             }
+          }
+          if constexpr (kBias) {
+            fill_bias(buf);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) release_tmem(buf);     // TMEM free for the MMA
           }
           ++kcount;
         }
@@ -393,15 +492,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if constexpr (RC == 32) tmem_ld32(taddr, r);
             else tmem_ld16(taddr + RC * c, r);
             tmem_ld_wait();
-            if (c == CW / RC - 1) {
+            if (!kBias && c == CW / RC - 1) {
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));   // TMEM free for the MMA
+              if (lane == 0) release_tmem(buf);   // TMEM free for the MMA
             }
 #pragma unroll
             for (int i = 0; i < RC / 2; ++i) {
               float x0, x1;
-              if constexpr (DT == kInt8) {
+              if constexpr (kBias) {
+                x0 = __uint_as_float(r[2 * i]) - kMagic;
+                x1 = __uint_as_float(r[2 * i + 1]) - kMagic;
+              } else if constexpr (DT == kInt8) {
                 x0 = __uint_as_float(r[2 * i] + kMagicBits) - kMagic;
                 x1 = __uint_as_float(r[2 * i + 1] + kMagicBits) - kMagic;
               } else {
@@ -411,6 +513,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               accf[RC * c + 2 * i] = fmaf(x0, f, accf[RC * c + 2 * i]);
               accf[RC * c + 2 * i + 1] = fmaf(x1, f, accf[RC * c + 2 * i + 1]);
             }
+          }
+          if constexpr (kBias) {
+            // refill after the last chunk is promoted (its registers are free)
+            fill_bias(buf);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) release_tmem(buf);     // TMEM free for the MMA
           }
           ++kcount;
         }
@@ -494,7 +604,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
       if (row_ok && n0 < p.N && p.out_f32) {
         float* frow = p.out_f32 + m * p.ldo + n0;
-        if (n0 + CW <= p.N && ((reinterpret_cast<uintptr_t>(frow) & 15) == 0)) {
+        if (n0 + CW <= p.N && ((reinterpret_cast<uintptr_t>(frow) & 31) == 0)) {
+#pragma unroll
+          for (int j = 0; j < CW; j += 8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h) w[h] = __float_as_uint(accf[j + h]);
+            st_global_v8(frow + j, w);
+          }
+        } else if (n0 + CW <= p.N && ((reinterpret_cast<uintptr_t>(frow) & 15) == 0)) {
 #pragma unroll
           for (int j = 0; j < CW; j += 4)
             *reinterpret_cast<float4*>(frow + j) =
@@ -508,7 +626,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         uint16_t* orow = p.out + m * p.ldo + n0;
         const bool full_n = n0 + CW <= p.N;
         const bool vec = full_n && ((reinterpret_cast<uintptr_t>(orow) & 15) == 0);
-        if (vec) {
+        if (vec && (reinterpret_cast<uintptr_t>(orow) & 31) == 0) {
+          // 32-byte stores: 16 outputs each, a full L2 sector per lane
+#pragma unroll
+          for (int j = 0; j < CW; j += 16) {
+            uint32_t w[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+              float v0 = accf[j + 2 * h];
+              float v1 = accf[j + 2 * h + 1];
+              if (p.bias) {
+                v0 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h));
+                v1 += bf16_bits_to_float(__ldg(p.bias + n0 + j + 2 * h + 1));
+              }
+              w[h] = (uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16);
+            }
+            st_global_v8(orow + j, w);
+          }
+        } else if (vec) {
 #pragma unroll
           for (int j = 0; j < CW; j += 8) {
             uint32_t w[4];
@@ -540,21 +675,50 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 
   tc_fence_before();
-  __syncthreads();
+  // neither CTA of a pair leaves (freeing shared memory that a pair MMA,
+  // load or arrive may still address) before the other is done
+  if constexpr (PAIR) cluster_sync_all();
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTBufs * BN);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, kTBufs * BN);
+    else tmem_dealloc(tmem_base, kTBufs * BN);
   }
 }
 
-template <int DT, int BN, int S, bool ONEK, bool SILU = false>
+// Clusters of two CTAs of a pair kernel the device holds at once.
+template <typename K>
+int max_active_pairs(K kern, uint32_t smem_bytes) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeClusterDimension;
+  at.val.clusterDim.x = 2;
+  at.val.clusterDim.y = 1;
+  at.val.clusterDim.z = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  return n;
+}
+
+template <int DT, int BN, int S, bool ONEK, bool SILU, bool PAIR>
 cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
-  using L = Smem<BN, S>;
-  auto kern = gemm_tc_kernel<DT, BN, S, ONEK, SILU>;
+  using L = Smem<BN, S, PAIR>;
+  constexpr int TM = PAIR ? 2 * BM : BM;
+  auto kern = gemm_tc_kernel<DT, BN, S, ONEK, SILU, PAIR>;
   static bool attr_set[64] = {};
+  static int pairs[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)L::kTotal);
     if (e != cudaSuccess) return e;
@@ -564,12 +728,13 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
     e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * kThreads < kSplitRegs) return cudaErrorInvalidConfiguration;
+    if (PAIR) pairs[dev] = max_active_pairs(kern, L::kTotal);
     attr_set[dev] = true;
   }
   CUtensorMap tA, tB;
   if (!make_tmap(&tA, a.qa, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.lda, BM) ||
       !make_tmap(&tB, a.qw, (uint64_t)a.K, (uint64_t)(a.N * a.E), (uint64_t)a.ldw,
-                 SILU ? 128u : (uint32_t)BN))
+                 SILU ? 128u : (uint32_t)(PAIR ? BN / 2 : BN)))
     return cudaErrorInvalidValue;
   TcParams p;
   p.sa = a.sa; p.sa_rows = a.sa_rows;
@@ -586,11 +751,39 @@ cudaError_t launch_typed(const GemmArgs& a, cudaStream_t st) {
   p.q_out = static_cast<uint8_t*>(a.q_out); p.ldq = a.ldq; p.s_out = a.s_out;
   p.out_f32 = a.out_f32;
   p.comb_acc = a.comb_acc; p.comb_perm = a.comb_perm; p.comb_w = a.comb_w; p.topk = (int)a.topk;
-  const int64_t mblk_bound = (a.M + BM - 1) / BM + (a.offsets ? a.E : 0);
+  const int64_t mblk_bound = (a.M + TM - 1) / TM + (a.offsets ? a.E : 0);
   const int64_t tiles_bound = mblk_bound * p.nblk;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles_bound, sm_count()));
-  kern<<<grid, kThreads, L::kTotal, st>>>(tA, tB, p);
-  return cudaGetLastError();
+  if (!PAIR) {
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles_bound, sm_count()));
+    kern<<<grid, kThreads, L::kTotal, st>>>(tA, tB, p);
+    return cudaGetLastError();
+  }
+  const int64_t npairs = std::max<int64_t>(1, std::min<int64_t>(tiles_bound, pairs[dev]));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * npairs), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kTotal;
+  cfg.stream = st;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeClusterDimension;
+  at.val.clusterDim.x = 2;
+  at.val.clusterDim.y = 1;
+  at.val.clusterDim.z = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tA, tB, p);
+}
+
+// Tile shape (tc_shape 1 forces one CTA per 128 x 256 tile, 2 a CTA pair per
+// 256 x 256 tile).  By size: measured on B200, the pair is faster with one
+// scale block along K (per-channel: 2020 against 1960 TOPS at 4096 x 14336 x
+// 4096) and slower with per-K-block promotion (block-wise INT8 1213 against
+// 1268 TOPS, FP8 1541 against 1585 TFLOPS), where the epilogue's TMEM
+// hand-off, not the operand feed the pair halves, sets the pace.
+bool use_pair(const GemmArgs& a) {
+  if (a.tc_shape == 1) return false;
+  if (a.tc_shape == 2) return true;
+  return a.bk >= a.K && a.M >= 512;
 }
 
 }  // namespace
@@ -634,8 +827,11 @@ bool tc_silu_supported(const GemmArgs& a, char* why, size_t n) {
 
 cudaError_t launch_gemm_tc_silu(const GemmArgs& a, cudaStream_t st) {
   if (a.M == 0 || a.seam == 0) return cudaSuccess;
-  if (a.dtype == kInt8) return launch_typed<kInt8, 256, 4, false, true>(a, st);
-  return launch_typed<kFp8, 256, 4, false, true>(a, st);
+  if (use_pair(a))
+    return a.dtype == kInt8 ? launch_typed<kInt8, 256, 6, false, true, true>(a, st)
+                            : launch_typed<kFp8, 256, 6, false, true, true>(a, st);
+  if (a.dtype == kInt8) return launch_typed<kInt8, 256, 4, false, true, false>(a, st);
+  return launch_typed<kFp8, 256, 4, false, true, false>(a, st);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
@@ -647,14 +843,25 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   // a single scale block along K (per-token / per-channel scales): promote
   // once per tile instead of once per 128-wide K-block
   const bool onek = a.bk >= a.K;
+  if (a.N > 128 && use_pair(a)) {
+    if (a.dtype == kInt8)
+      return onek ? launch_typed<kInt8, 256, 6, true, false, true>(a, st)
+                  : launch_typed<kInt8, 256, 6, false, false, true>(a, st);
+    return onek ? launch_typed<kFp8, 256, 6, true, false, true>(a, st)
+                : launch_typed<kFp8, 256, 6, false, false, true>(a, st);
+  }
   if (a.N > 128) {
     if (a.dtype == kInt8)
-      return onek ? launch_typed<kInt8, 256, 4, true>(a, st) : launch_typed<kInt8, 256, 4, false>(a, st);
-    return onek ? launch_typed<kFp8, 256, 4, true>(a, st) : launch_typed<kFp8, 256, 4, false>(a, st);
+      return onek ? launch_typed<kInt8, 256, 4, true, false, false>(a, st)
+                  : launch_typed<kInt8, 256, 4, false, false, false>(a, st);
+    return onek ? launch_typed<kFp8, 256, 4, true, false, false>(a, st)
+                : launch_typed<kFp8, 256, 4, false, false, false>(a, st);
   }
   if (a.dtype == kInt8)
-    return onek ? launch_typed<kInt8, 128, 6, true>(a, st) : launch_typed<kInt8, 128, 6, false>(a, st);
-  return onek ? launch_typed<kFp8, 128, 6, true>(a, st) : launch_typed<kFp8, 128, 6, false>(a, st);
+    return onek ? launch_typed<kInt8, 128, 6, true, false, false>(a, st)
+                : launch_typed<kInt8, 128, 6, false, false, false>(a, st);
+  return onek ? launch_typed<kFp8, 128, 6, true, false, false>(a, st)
+              : launch_typed<kFp8, 128, 6, false, false, false>(a, st);
 }
 
 }  // namespace bq

@@ -239,27 +239,44 @@ cudaError_t launch_moe_combine(const void* y, int64_t ldy, const int32_t* inv_pe
 
 // out[t, n] = bf16(acc[t, n]) and acc[t, n] = 0: the single rounding of
 // the combine sums the w2 epilogue accumulated, leaving the sums ready for
-// the next layer call.  Four columns per thread.
+// the next layer call.  Four columns per chunk; a thread first loads its
+// kFinUnroll chunks, then stores them: a store of zeros right behind the
+// load of the same address holds the thread's next load until the first
+// returns (measured on B200: 6.5x slower at 64 MB of sums).
+constexpr int kFinUnroll = 8;
+
 __global__ void __launch_bounds__(256)
 moe_combine_finish_kernel(float* __restrict__ acc, int64_t T, int64_t N, int64_t ld_acc,
                           uint16_t* __restrict__ out, int64_t ldo, bool vec) {
   const int64_t chunks = (N + 3) / 4;
   const int64_t total = T * chunks;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = idx / chunks, n0 = (idx - t * chunks) * 4;
-    float* a = acc + t * ld_acc + n0;
-    uint16_t* o = out + t * ldo + n0;
-    if (vec && n0 + 4 <= N) {
-      const float4 v = *reinterpret_cast<const float4*>(a);
-      *reinterpret_cast<float4*>(a) = make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<uint2*>(o) =
-          make_uint2((uint32_t)float_to_bf16_bits(v.x) | ((uint32_t)float_to_bf16_bits(v.y) << 16),
-                     (uint32_t)float_to_bf16_bits(v.z) | ((uint32_t)float_to_bf16_bits(v.w) << 16));
-    } else {
-      for (int i = 0; i < 4 && n0 + i < N; ++i) {
-        o[i] = float_to_bf16_bits(a[i]);
-        a[i] = 0.f;
+  const int64_t tile = (int64_t)blockDim.x * kFinUnroll;
+  for (int64_t base = (int64_t)blockIdx.x * tile; base < total; base += (int64_t)gridDim.x * tile) {
+    float4 v[kFinUnroll];
+#pragma unroll
+    for (int k = 0; k < kFinUnroll; ++k) {
+      const int64_t idx = base + (int64_t)k * blockDim.x + threadIdx.x;
+      if (idx >= total) break;
+      const int64_t t = idx / chunks, n0 = (idx - t * chunks) * 4;
+      if (vec && n0 + 4 <= N) v[k] = *reinterpret_cast<const float4*>(acc + t * ld_acc + n0);
+    }
+#pragma unroll
+    for (int k = 0; k < kFinUnroll; ++k) {
+      const int64_t idx = base + (int64_t)k * blockDim.x + threadIdx.x;
+      if (idx >= total) break;
+      const int64_t t = idx / chunks, n0 = (idx - t * chunks) * 4;
+      float* a = acc + t * ld_acc + n0;
+      uint16_t* o = out + t * ldo + n0;
+      if (vec && n0 + 4 <= N) {
+        *reinterpret_cast<float4*>(a) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<uint2*>(o) = make_uint2(
+            (uint32_t)float_to_bf16_bits(v[k].x) | ((uint32_t)float_to_bf16_bits(v[k].y) << 16),
+            (uint32_t)float_to_bf16_bits(v[k].z) | ((uint32_t)float_to_bf16_bits(v[k].w) << 16));
+      } else {
+        for (int i = 0; i < 4 && n0 + i < N; ++i) {
+          o[i] = float_to_bf16_bits(a[i]);
+          a[i] = 0.f;
+        }
       }
     }
   }
@@ -271,7 +288,8 @@ cudaError_t launch_moe_combine_finish(float* acc, int64_t T, int64_t N, int64_t 
   const bool vec = ((uintptr_t)acc % 16 == 0) && ((uintptr_t)out % 8 == 0) && ld_acc % 4 == 0 &&
                    ldo % 4 == 0;
   const int64_t total = T * ((N + 3) / 4);
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, 148 * 8));
+  const int64_t tiles = (total + 256 * kFinUnroll - 1) / (256 * kFinUnroll);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, 148 * 8));
   moe_combine_finish_kernel<<<grid, 256, 0, st>>>(acc, T, N, ld_acc, static_cast<uint16_t*>(out),
                                                   ldo, vec);
   return cudaGetLastError();

@@ -97,6 +97,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// One 32-byte (256-bit) global store from a thread; p 32-byte aligned.  A
+// full L2 sector per lane, half the store instructions of 16-byte stores.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// Ask L2 to fetch a 2-D tile of the tensor map (no shared-memory copy).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // L2 policy for data read exactly once (streamed weights): evict it first, so
 // it does not push small, reused tensors (activations, scales, outputs) out.
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -208,6 +224,14 @@ __device__ __forceinline__ void tmem_st32_fill(uint32_t taddr, uint32_t v) {
       : "memory");
 }
 
+// 32 lanes x 4 columns store; every column gets the value v (the source is
+// a range of 4 registers, so the narrow form keeps register pressure low).
+__device__ __forceinline__ void tmem_st4_fill(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr),
+               "r"(v)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -281,6 +305,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster with the default
+// (release, CTA-scope) semantics: the signal a pair's epilogue gives the
+// leader's MMA, whose TMEM hand-off is ordered by the tcgen05 fences.  The
+// cluster-scope release of mbar_arrive_cluster costs far more per arrive.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2-D tile load into this CTA's shared memory whose completion is counted on

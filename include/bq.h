@@ -85,9 +85,10 @@ typedef enum bq_dtype {
 typedef enum bq_path {
     BQ_PATH_AUTO = 0,     /* choose by shape and alignment */
     BQ_PATH_SIMT = 1,     /* generic CUDA-core kernel: any shape/stride */
-    BQ_PATH_TCGEN05 = 2,  /* TMA + tcgen05 tensor-core kernel (large M) */
+    BQ_PATH_TCGEN05 = 2,  /* TMA + tcgen05 tensor-core kernel (large M; tile shape by size) */
     BQ_PATH_DECODE = 3,   /* split-K weight-streaming kernel (small M) */
-    BQ_PATH_TCGEN05_1CTA = 4   /* force the tcgen05 kernel (128x256 tiles) */
+    BQ_PATH_TCGEN05_1CTA = 4,  /* force the single-CTA tcgen05 kernel (128x256 tiles) */
+    BQ_PATH_TCGEN05_PAIR = 5   /* force the CTA-pair tcgen05 kernel (256x256 tiles, cta_group::2) */
 } bq_path;
 
 /* ---- library information and errors ---------------------------------- */
@@ -358,7 +359,7 @@ bq_status bq_grouped_gemm(const void* qa, int64_t lda, const float* sa, int64_t 
  * q: codes [R, I] (row stride ldq, a multiple of 16; q 16-byte aligned),
  * s: fp32 [I/128][R].  Rows past expert_offsets[E] are left untouched.
  * Needs block_n = block_k = 128, I a multiple of 128, and the tensor-core
- * path (BQ_PATH_AUTO, BQ_PATH_TCGEN05 or BQ_PATH_TCGEN05_1CTA); otherwise
+ * path (BQ_PATH_AUTO or one of the BQ_PATH_TCGEN05 paths); otherwise
  * BQ_ERR_UNSUPPORTED, and the caller runs the two unfused calls.  Needs no
  * workspace. */
 bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* sa, int64_t R,
@@ -387,7 +388,7 @@ bq_status bq_grouped_gemm_silu_quant(const void* qa, int64_t lda, const float* s
  * recorded in the device status word as BQ_ERR_INVALID_ARG); topk_w: fp32
  * [T, topk].  Rows past expert_offsets[E] add nothing.  Needs R a multiple
  * of topk, block_n = block_k = 128 (or block_k >= K) and the tensor-core
- * path (BQ_PATH_AUTO, BQ_PATH_TCGEN05 or BQ_PATH_TCGEN05_1CTA); otherwise
+ * path (BQ_PATH_AUTO or one of the BQ_PATH_TCGEN05 paths); otherwise
  * BQ_ERR_UNSUPPORTED.  Needs no workspace. */
 bq_status bq_grouped_gemm_combine(const void* qa, int64_t lda, const float* sa, int64_t R,
                                   const int32_t* expert_offsets, int64_t E, const void* qw,
@@ -438,7 +439,7 @@ bq_status bq_mx_quant_weight(const float* w, int64_t N, int64_t K, int64_t ldw, 
  * NULL; out bf16 [M, N] (row stride ldo).  Needs K a positive multiple of
  * 128, lda and ldw multiples of 16, and 16-byte aligned qa, qw, sfa, sfw
  * (else BQ_ERR_UNSUPPORTED / BQ_ERR_ALIGNMENT), and the tensor-core path
- * (BQ_PATH_AUTO, BQ_PATH_TCGEN05 or BQ_PATH_TCGEN05_1CTA).  No workspace. */
+ * (BQ_PATH_AUTO or one of the BQ_PATH_TCGEN05 paths).  No workspace. */
 bq_status bq_mx_gemm(const void* qa, int64_t lda, const void* sfa, const void* qw, int64_t ldw,
                      const void* sfw, int64_t M, int64_t N, int64_t K, const void* bias,
                      void* out, int64_t ldo, void* stream);

@@ -138,10 +138,11 @@ TC_SHAPES = [
     (257, 640, 2048),
     (64, 1280, 384),
     (1000, 384, 4096),
+    (513, 768, 640),      # a CTA pair's 256-row tiles: one row past two of them
 ]
 
 
-@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA])
+@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_PAIR])
 @pytest.mark.parametrize("dtype", [INT8, FP8])
 @pytest.mark.parametrize("M,N,K", TC_SHAPES)
 def test_gemm_tcgen05_vs_oracle(path, dtype, M, N, K):
@@ -421,7 +422,7 @@ def test_moe_layer_stages_vs_oracle():
     assert_combine_close(out, oracle.moe_combine(yb, i_ref, p["tw"]), yb, i_ref, p["tw"])
 
 
-@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA])
+@pytest.mark.parametrize("path", [bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_PAIR])
 @pytest.mark.parametrize("dtype", [INT8, FP8])
 def test_grouped_gemm_tcgen05_vs_oracle(path, dtype):
     p = moe_problem(T=300, H=384, I=256, E=8, dtype=dtype, seed=33)
@@ -439,6 +440,56 @@ def test_grouped_gemm_tcgen05_vs_oracle(path, dtype):
     ref13 = oracle.grouped_gemm(qx[rows], sx[rows], o_ref, p["q13"], p["s13"], 128, 128, dtype,
                                 seam=I)
     assert_gemm_close(y13, ref13, "tcgen05 grouped w13")
+
+
+@pytest.mark.parametrize("dtype", [INT8, FP8])
+def test_cta_pair_and_single_cta_kernels_agree_bit_for_bit(dtype):
+    """The CTA-pair kernel (256-row tiles, cta_group::2 MMAs) and the
+    single-CTA kernel sum the same K-blocks in the same order and promote
+    them identically: every output is the same bits.  Dense with bias (M and
+    N ragged against 256, a partial last K-block), one scale block along K,
+    the grouped w13 with its gate/up seam, the fused SiLU requantisation and
+    the combining w2."""
+    def both(fn):
+        outs = []
+        for path in (bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_PAIR):
+            bq.set_path(path)
+            outs.append(fn())
+        bq.set_path(bq.PATH_AUTO)
+        torch.cuda.synchronize()
+        bq.check_device_status()
+        return outs
+
+    def same(a, b, what):
+        a = a if isinstance(a, (tuple, list)) else (a,)
+        b = b if isinstance(b, (tuple, list)) else (b,)
+        for x, y in zip(a, b):
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), what
+
+    _, qa, sa, qw, sw, bb = make_problem(600, 640, 1008, 128, 128, dtype, 91, bias=True)
+    args = (dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), 128, 128, dtype)
+    same(*both(lambda: bq.gemm(*args, bias=dev_bf16(bb))), "dense")
+    same(*both(lambda: bq.gemm_partial(*args)), "dense fp32 partial")
+    xb = act_bits(520, 512, 92)
+    q1, s1 = oracle.quant_act(xb, 512, dtype)
+    qw1, sw1 = oracle.quant_weight(bq_synth.weights(768, 512, 0.02, 93).numpy(), 1, 512, dtype)
+    same(*both(lambda: bq.gemm(dev_u8(q1), dev_f32(s1.T), dev_u8(qw1), dev_f32(sw1), 1, 512,
+                               dtype)), "one scale block along K")
+    p = moe_problem(T=700, H=384, I=256, E=8, dtype=dtype, seed=94)
+    off, perm, inv = bq.moe_permute(dev_i32(p["ids"]), 8)
+    qg, sg = bq.moe_quant_gather(dev_bf16(p["x"]), perm, 2, 128, dtype)
+    q13, s13 = dev_u8(p["q13"]), dev_f32(p["s13"])
+    same(*both(lambda: bq.grouped_gemm(qg, sg, off, q13, s13, 128, 128, n_seam=256,
+                                       dtype=dtype)), "grouped w13")
+    (qh, sh), (qh2, sh2) = both(lambda: bq.grouped_gemm_silu_quant(qg, sg, off, q13, s13, dtype))
+    same((qh, sh), (qh2, sh2), "fused SiLU requantisation")
+    q2, s2, tw = dev_u8(p["q2"]), dev_f32(p["s2"]), dev_f32(p["tw"])
+
+    def comb():
+        acc = torch.zeros(700, 384, dtype=torch.float32, device="cuda")
+        bq.grouped_gemm_combine(qh, sh, off, q2, s2, perm, tw, acc, dtype)
+        return bq.moe_combine_finish(acc)
+    same(*both(comb), "combining w2")
 
 
 # w2 grouped GEMM fused with the weighted top-k combine
@@ -610,7 +661,7 @@ def test_fused_w13_silu_requant_rows_past_offsets_and_paths():
     bq.set_path(bq.PATH_AUTO)
 
 
-@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05_1CTA])
+@pytest.mark.parametrize("path", [bq.PATH_SIMT, bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_PAIR])
 def test_grouped_gemm_leaves_rows_past_offsets_untouched(path):
     p = moe_problem(T=50, H=128, I=128, E=4)
     bq.set_path(path)
@@ -662,7 +713,7 @@ ONEK_SHAPES = [(300, 512, 512, 1), (1024, 1000, 1000, 1), (260, 768, 4096, 128),
 
 @pytest.mark.parametrize("dtype", [INT8, FP8])
 @pytest.mark.parametrize("M,N,K,bn", ONEK_SHAPES)
-@pytest.mark.parametrize("path", [bq.PATH_AUTO, bq.PATH_TCGEN05_1CTA])
+@pytest.mark.parametrize("path", [bq.PATH_AUTO, bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_PAIR])
 def test_one_scale_block_along_k(path, M, N, K, bn, dtype):
     xb = act_bits(M, K, 500 + M, max(1, K // 100), 30.0)
     w = bq_synth.weights(N, K, 0.02, 501 + N).numpy()
@@ -680,7 +731,7 @@ def test_one_scale_block_along_k(path, M, N, K, bn, dtype):
     assert np.array_equal(swg.cpu().numpy().view(np.uint32), sw.view(np.uint32))
     bq.set_path(path)
     try:
-        if path == bq.PATH_TCGEN05_1CTA and K % 16 != 0:
+        if path in (bq.PATH_TCGEN05_1CTA, bq.PATH_TCGEN05_PAIR) and K % 16 != 0:
             # TMA rows must be multiples of 16 bytes: the forced path refuses
             with pytest.raises(bq.BqError) as ei:
                 bq.gemm(dev_u8(qa), dev_f32(sa.T), dev_u8(qw), dev_f32(sw), bn, K, dtype)

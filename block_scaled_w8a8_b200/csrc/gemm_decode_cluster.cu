@@ -115,6 +115,14 @@ __device__ __forceinline__ void named_bar_arrive(int id, int n) {
   asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Ask L2 to fetch a 2-D tile of the tensor map (no shared-memory copy).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to
 // another CTA's (cluster address), completion counted on the mbarrier at
 // cluster address `bar` in the destination CTA.

@@ -105,14 +105,6 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
                : "memory");
 }
 
-// Ask L2 to fetch a 2-D tile of the tensor map (no shared-memory copy).
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* m, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
 // L2 policy for data read exactly once (streamed weights): evict it first, so
 // it does not push small, reused tensors (activations, scales, outputs) out.
 __device__ __forceinline__ uint64_t policy_evict_first() {

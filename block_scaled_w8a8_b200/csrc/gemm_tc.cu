@@ -131,9 +131,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   // 12582912 + P_kb exactly (|P_kb| <= 128 * 127 * 127 < 2^22), so the
   // epilogue needs one FADD and one FFMA per element and no integer add; it
   // refills the buffer with the bias as it frees it.  Measured on B200: +8%
-  // on the block-wise INT8 GEMM (1176 -> 1268 TOPS at 4096 x 14336 x 4096),
-  // but -28% on the fused SiLU kernel (1349 -> 1873 us for the MoE w13),
-  // which therefore adds the bias with an integer add instead
+  // on the block-wise INT8 GEMM (1176 -> 1268 TOPS at 4096 x 14336 x 4096).
+  // The fused SiLU kernel adds the bias with an integer add, as before
   constexpr bool kBias = DT == kInt8 && !ONEK && !SILU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -457,7 +456,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const float f = c < 2 ? fg : fu;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float x = kBias ? __uint_as_float(r[i]) - kMagic : __uint_as_float(r[i]);
+              const float x = kBias            ? __uint_as_float(r[i]) - kMagic
+                              : DT == kInt8 ? __uint_as_float(r[i] + kMagicBits) - kMagic
+                                            : __uint_as_float(r[i]);
               accf[16 * c + i] = fmaf(x, f, accf[16 * c + i]);
             }
           }

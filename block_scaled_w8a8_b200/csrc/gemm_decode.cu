@@ -478,10 +478,17 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
       }
     }
-    return;
   }
-  // producer and MMA warps: complete their part of the start-up barrier
-  if (p.cluster) cluster_wait();
+  if (p.cluster) {
+    // producer and MMA warps: their part of the start-up barrier (the
+    // epilogue warps waited on it before pushing)
+    if (warp < 2) cluster_wait();
+    // every CTA of the cluster, aborted or not, meets here before exiting, so
+    // no peer still pushes into or arrives on this CTA's shared memory after
+    // it has gone (every wait before this one is bounded)
+    cluster_arrive();
+    cluster_wait();
+  }
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

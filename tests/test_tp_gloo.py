@@ -101,7 +101,7 @@ def _worker(rank, world, port, case, q):
         loc = OracleLocal(oracle)
         res = {}
         if case in ("column", "row"):
-            M, N, K = 19, 512, 768
+            M, N, K = 19, 512, _linear_k(world)
             x = bq_synth.activations(M, K, 3, 7, 20.0)
             w = bq_synth.weights(N, K, 0.02, 4).numpy()
             bias = bq_synth.activations(1, N, 5)[0]
@@ -120,8 +120,9 @@ def _worker(rank, world, port, case, q):
                     qw[:, rank * k:(rank + 1) * k].contiguous(),
                     sw[:, rank * k // 128:(rank + 1) * k // 128].contiguous(), bias,
                     group=None, local=loc)
+                ms = _scatter_rows(world)
                 y2 = tp.row_parallel_linear(
-                    x[:18, rank * k:(rank + 1) * k].contiguous(),
+                    x[:ms, rank * k:(rank + 1) * k].contiguous(),
                     qw[:, rank * k:(rank + 1) * k].contiguous(),
                     sw[:, rank * k // 128:(rank + 1) * k // 128].contiguous(), bias,
                     group=None, scatter_rows=True, local=loc)
@@ -161,6 +162,16 @@ def _worker(rank, world, port, case, q):
         q.put((rank, None, traceback.format_exc()))
 
 
+def _linear_k(world):
+    """K of the linear cases: K / world must be a whole number of 128-blocks."""
+    return 768 if world == 2 else 1024
+
+
+def _scatter_rows(world):
+    """Token rows of the reduce-scatter case: a multiple of the group size."""
+    return 18 if world == 2 else 16
+
+
 def _run(case, world=2):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -178,10 +189,10 @@ def _run(case, world=2):
     return out
 
 
-def _reference_linear():
+def _reference_linear(world=2):
     import bq_synth
     import oracle
-    M, N, K = 19, 512, 768
+    M, N, K = 19, 512, _linear_k(world)
     x = bq_synth.activations(M, K, 3, 7, 20.0)
     w = bq_synth.weights(N, K, 0.02, 4).numpy()
     bias = _bits(bq_synth.activations(1, N, 5)[0])
@@ -211,7 +222,6 @@ def test_row_parallel_rounds_once_after_the_fp32_sum():
         ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref64), 1e-30))) - 7)
         assert np.all(np.abs(d) <= ulp + 1e-30)
         # the reduce-scatter form leaves rank r the rows [9 r, 9 r + 9)
-        sc = oracle.bf16_to_f64(out[rank]["scattered"])
         assert np.array_equal(out[rank]["scattered"], out[rank]["y"][9 * rank:9 * rank + 9])
 
 
@@ -228,3 +238,25 @@ def test_partition_rule_rejects_cut_blocks():
         tp.check_partition(2, 1024, 512, [200, 312])       # output shard not a block_n multiple
     with pytest.raises(BqError):
         tp.check_partition(2, 640, 320, [256])              # input shard not a block_k multiple
+
+
+def test_four_ranks():
+    """The same three forms over four gloo ranks: column and expert parallel
+    (one expert per rank, so some ranks receive no rows from others) equal the
+    unsharded layer bit for bit; row parallel sums four fp32 partials and
+    rounds once (within one bf16 ulp), and its reduce-scatter leaves rank r
+    rows [4 r, 4 r + 4)."""
+    import oracle
+    ref64 = _reference_linear(4)
+    out = _run("column", world=4)
+    for rank in range(4):
+        assert np.array_equal(out[rank]["y"], oracle.bf16_from_f64(ref64))
+    out = _run("row", world=4)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref64), 1e-30))) - 7)
+    for rank in range(4):
+        d = oracle.bf16_to_f64(out[rank]["y"]) - ref64
+        assert np.all(np.abs(d) <= ulp + 1e-30)
+        assert np.array_equal(out[rank]["scattered"], out[rank]["y"][4 * rank:4 * rank + 4])
+    out = _run("moe", world=4)
+    for rank in range(4):
+        assert np.array_equal(out[rank]["y"], out[rank]["ref"])

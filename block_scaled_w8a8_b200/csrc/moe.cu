@@ -136,8 +136,10 @@ moe_combine_kernel(const uint16_t* __restrict__ y, int64_t ldy,
   }
 }
 
-// Waits for a flag that nothing sets, at most spin_limit polls, then records
-// a timeout in the status word and returns.
+// Top-k routing of one token per warp: the k largest logits in k rounds of a
+// warp arg-max (ties to the lower expert index; softmax is increasing, so
+// this is the top-k of the probabilities), then their softmax weights
+// renormalised over the k: exp(l_j - l_max) / sum.
 constexpr int kRouteMaxE = 256, kRouteMaxK = 8;
 
 __global__ void __launch_bounds__(256)
@@ -196,6 +198,8 @@ moe_route_kernel(const float* __restrict__ logits, int64_t ld, int64_t T, int E,
   }
 }
 
+// Waits for a flag that nothing sets, at most spin_limit polls, then records
+// a timeout in the status word and returns.
 __global__ void selftest_wait_kernel(int64_t spin_limit, unsigned* status) {
   __shared__ volatile int flag;
   if (threadIdx.x == 0) flag = 0;

@@ -144,7 +144,43 @@ def test_quant_and_moe_argument_errors_on_host(L):
     assert bq.mx_scale_bytes(300, 512) == 3 * 4 * 512
     assert L.bq_set_path(9) == bq.ERR_INVALID_ARG
     assert L.bq_set_path(7) == bq.ERR_INVALID_ARG
+    assert L.bq_set_path(6) == bq.ERR_INVALID_ARG
+    assert L.bq_set_path(bq.PATH_TCGEN05_PAIR) == bq.OK
+    assert L.bq_set_path(bq.PATH_AUTO) == bq.OK
     assert L.bq_selftest_bounded_wait(0, None) == bq.ERR_INVALID_ARG
+
+
+def test_routing_combine_and_partial_argument_errors_on_host(L):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # routing: topk > E, ld < E, E beyond 256, topk beyond 8; T = 0 is a no-op
+    assert L.bq_moe_route(fake, 8, 4, 8, 9, fake, fake, None) == bq.ERR_INVALID_ARG
+    assert L.bq_moe_route(fake, 4, 4, 8, 2, fake, fake, None) == bq.ERR_INVALID_ARG
+    assert L.bq_moe_route(fake, 300, 4, 300, 2, fake, fake, None) == bq.ERR_UNSUPPORTED
+    assert L.bq_moe_route(fake, 16, 4, 16, 9, fake, fake, None) == bq.ERR_UNSUPPORTED
+    assert L.bq_moe_route(None, 8, 0, 8, 2, None, None, None) == bq.OK
+    # the combining w2 GEMM: topk 0, R not T * topk, ld_acc < N, and a path
+    # that is not a tensor-core one; R = 0 is a no-op
+    args = (fake, 128, fake, 9, fake, 2, fake, fake, 256, 128, 128, 128, 0, fake, fake)
+    assert L.bq_grouped_gemm_combine(*args, 0, fake, 256, None) == bq.ERR_INVALID_ARG
+    assert L.bq_grouped_gemm_combine(*args, 2, fake, 256, None) == bq.ERR_INVALID_ARG
+    args8 = (fake, 128, fake, 8, fake, 2, fake, fake, 256, 128, 128, 128, 0, fake, fake)
+    assert L.bq_grouped_gemm_combine(*args8, 2, fake, 128, None) == bq.ERR_INVALID_ARG
+    L.bq_set_path(bq.PATH_SIMT)
+    try:
+        assert L.bq_grouped_gemm_combine(*args8, 2, fake, 256, None) == bq.ERR_UNSUPPORTED
+    finally:
+        L.bq_set_path(bq.PATH_AUTO)
+    assert L.bq_grouped_gemm_combine(None, 128, None, 0, fake, 2, None, None, 256, 128, 128,
+                                     128, 0, None, None, 2, None, 256, None) == bq.OK
+    # the finishing passes: leading dimensions below N; empty problems
+    assert L.bq_moe_combine_finish(fake, 4, 256, 128, fake, 256, None) == bq.ERR_INVALID_ARG
+    assert L.bq_moe_combine_finish(None, 0, 256, 256, None, 256, None) == bq.OK
+    assert L.bq_finish_bf16(fake, 128, 4, 256, None, fake, 256, None) == bq.ERR_INVALID_ARG
+    assert L.bq_finish_bf16(None, 256, 0, 256, None, None, 256, None) == bq.OK
+    # the fp32 partial GEMM: an output stride below N
+    assert L.bq_gemm_partial(fake, 128, fake, fake, 128, fake, 4, 256, 128, 128, 128, 0,
+                             fake, 128, None, 0, None) == bq.ERR_INVALID_ARG
 
 
 def test_workspace_queries_are_host_only(L):
